@@ -1,0 +1,113 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU parity tests and bench.py.
+
+This module only draws numbers.  It holds none of the attention arithmetic: no
+masks, no softmax, no cache bookkeeping.  Both sides of every parity check (the
+float64 oracle under ``oracle/`` and the CUDA library) read the tensors returned
+here, so they see bit-identical inputs.
+
+Workload shapes follow the pages' examples:
+  * lingbot-map frames are 518x378 images at patch 14 -> 37*27 = 999 patch tokens
+    plus 1 camera and 4 register tokens, P = 1004 tokens per frame, C = 1024,
+    16 heads of 64 (AggregatorStream guide; FlashInferBlock.forward signature,
+    ``num_register_tokens=4``);
+  * the Mistral-style token window is W = 4096 with grouped-query attention
+    (sliding-window attention explainer, Mistral 7B paragraph).
+
+All generators use ``torch.Generator('cpu')`` so the values do not depend on the
+GPU.  bf16 tensors are produced by rounding a float32 draw to bfloat16 (round to
+nearest even, torch's ``.to``).
+"""
+from __future__ import annotations
+
+import torch
+
+# ---------------------------------------------------------------- constants
+P_FRAME = 1004          # 1 camera + 4 register + 37*27 patch tokens
+NUM_SPECIAL = 5         # camera + 4 register tokens lead every frame
+C_MODEL = 1024
+HEADS = 16
+HEAD_DIM = 64
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def normal(shape, seed: int, dtype=torch.float32) -> torch.Tensor:
+    """i.i.d. N(0,1) draw, rounded to ``dtype``."""
+    x = torch.randn(*shape, generator=_gen(seed), dtype=torch.float32)
+    return x.to(dtype)
+
+
+def tiny_qkv(seed: int = 0, B: int = 1, F: int = 8, P: int = 21, H: int = 2, D: int = 32,
+             dtype=torch.float32):
+    """Tiny check workload: q, k, v ~ N(0,1) of shape [B, F*P, H, D].
+
+    Default shape: 8 frames of 21 tokens (1 camera + 4 register + 16 patch),
+    2 heads of 32, float32.
+    """
+    g = _gen(seed)
+    shape = (B, F * P, H, D)
+    q = torch.randn(*shape, generator=g, dtype=torch.float32).to(dtype)
+    k = torch.randn(*shape, generator=g, dtype=torch.float32).to(dtype)
+    v = torch.randn(*shape, generator=g, dtype=torch.float32).to(dtype)
+    return q, k, v
+
+
+def projected_qkv(seed: int = 0, F: int = 32, P: int = P_FRAME, C: int = C_MODEL,
+                  H: int = HEADS, std: float = 0.02, dtype=torch.bfloat16):
+    """Prefill workload: Q/K/V = LayerNorm(x) @ W_{q,k,v}, x ~ N(0,1) [F*P, C],
+    W ~ N(0, std^2) [C, C]; LayerNorm without affine parameters, eps 1e-5.
+
+    Returns q, k, v of shape [1, F*P, H, C//H] in ``dtype``.  The projection is
+    input synthesis (it shapes the value distribution like a real layer's),
+    not part of the attention path.
+    """
+    g = _gen(seed)
+    N = F * P
+    x = torch.randn(N, C, generator=g, dtype=torch.float32)
+    w = [torch.randn(C, C, generator=g, dtype=torch.float32) * std for _ in range(3)]
+    x = torch.nn.functional.layer_norm(x, (C,), eps=1e-5)
+    out = []
+    for wi in w:
+        y = (x @ wi).reshape(1, N, H, C // H).to(dtype)
+        out.append(y.contiguous())
+    return tuple(out)
+
+
+def stream_frame(frame_idx: int, P: int = P_FRAME, H: int = HEADS, D: int = HEAD_DIM,
+                 dtype=torch.bfloat16, base_seed: int = 0):
+    """One streaming frame: q, k, v ~ N(0,1) of shape [P, H, D], seeded by the
+    frame index (plus ``base_seed`` so layers can differ)."""
+    g = _gen(base_seed * 1_000_003 + frame_idx)
+    q = torch.randn(P, H, D, generator=g, dtype=torch.float32).to(dtype)
+    k = torch.randn(P, H, D, generator=g, dtype=torch.float32).to(dtype)
+    v = torch.randn(P, H, D, generator=g, dtype=torch.float32).to(dtype)
+    return q, k, v
+
+
+def band_qkv(seed: int = 1, N: int = 32768, Hq: int = 32, Hkv: int = 8, D: int = 128,
+             dtype=torch.bfloat16):
+    """Token-window GQA prefill workload: Q [1,N,Hq,D], K,V [1,N,Hkv,D] ~ N(0,1)."""
+    g = _gen(seed)
+    q = torch.randn(1, N, Hq, D, generator=g, dtype=torch.float32).to(dtype)
+    k = torch.randn(1, N, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    v = torch.randn(1, N, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    return q, k, v
+
+
+def decode_inputs(seed: int = 1, B: int = 64, W: int = 4096, Hq: int = 32, Hkv: int = 8,
+                  D: int = 128, dtype=torch.bfloat16):
+    """Single-token GQA decode workload against a fully populated rolling cache.
+
+    Returns q [B,Hq,D], k_new, v_new [B,Hkv,D], k_cache, v_cache [B,W,Hkv,D].
+    """
+    g = _gen(seed)
+    k_cache = torch.randn(B, W, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    v_cache = torch.randn(B, W, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    q = torch.randn(B, Hq, D, generator=g, dtype=torch.float32).to(dtype)
+    k_new = torch.randn(B, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    v_new = torch.randn(B, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
+    return q, k_new, v_new, k_cache, v_cache
