@@ -1,0 +1,231 @@
+/*
+ * swa.h -- C ABI of the B200 (sm_100a) frame-causal sliding-window attention library.
+ *
+ * One shared library, libswa_b200.so, exports every function below with C linkage.
+ * Signatures carry only plain pointers, integers and sizes.  Tensor pointers are
+ * DEVICE pointers owned by the caller unless a comment says otherwise; the library
+ * never frees or retains them beyond the call.  ``stream`` is a cudaStream_t passed
+ * as void* (NULL = the legacy default stream); every call is asynchronous on it
+ * unless documented as synchronous.  Calls validate their arguments on the host and
+ * return a negative swa_status before launching anything when they are invalid.
+ *
+ * Method sources (page title, section):
+ *   [AGG] "Sliding Window Attention Mechanism in AggregatorStream: Implementation and
+ *         Configuration Guide": "Mask Generation in CausalAttention" (window start
+ *         max(0, i - sliding_window_size*num_frame_per_block + 1), ANDed with the
+ *         causal mask), "KV Cache Eviction Strategy" (evict before attention; the
+ *         first scale frames stay; special tokens can persist), FAQ on
+ *         sliding_window_size = -1 (full causal).
+ *   [IO]  "Stream.py Aggregator Input and Output Formats": tokens [B*S, P, C],
+ *         scalar parameters B, S, P, C, global_idx, num_frame_for_scale,
+ *         sliding_window_size.
+ *   [BLK] "Method forward" (lingbot_map/layers/block.py FlashInferBlock.forward):
+ *         the streaming step append_frame -> evict_frames -> compute_attention on
+ *         per-frame q/k/v of shape [tpf, H, D]; global_idx selects the block's cache.
+ *   [SWA] sliding-window attention explainer (Mistral 7B): token band i-W+1..i,
+ *         rolling KV buffer written at slot i mod W, grouped-query attention.
+ *
+ * Numerics: bf16 inputs and outputs with float32 accumulation and softmax on the
+ * tensor-core path (head_dim 64 or 128); float32 end to end on the SIMT path
+ * (head_dim 32, 64 or 128).  The softmax scale is 1/sqrt(head_dim).
+ */
+#ifndef SWA_B200_H
+#define SWA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status */
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_ARG = -1,         /* null pointer, bad enum, negative size            */
+    SWA_ERR_SHAPE = -2,       /* inconsistent sizes, e.g. C != heads*head_dim      */
+    SWA_ERR_ORDER = -3,       /* streaming frame out of order / attend before append */
+    SWA_ERR_CAPACITY = -4,    /* buffer too small, cache full, layer out of range  */
+    SWA_ERR_CUDA = -5,        /* a CUDA runtime call failed                        */
+    SWA_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (latched flag) */
+    SWA_ERR_UNSUPPORTED = -7  /* dtype / head_dim combination not built            */
+} swa_status;
+
+typedef enum { SWA_F32 = 0, SWA_BF16 = 1 } swa_dtype;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* swa_status_str(int status);
+
+/* Library ABI version (major*100 + minor). */
+int swa_version(void);
+
+/* ------------------------------------------------------------ tile scheduler
+ * Host-side views of the block-sparse schedule the kernels use (the device code
+ * runs the same functions).  Intended for tests and tooling; no GPU needed.
+ *
+ * swa_sched_frame_intervals: key-frame intervals visible to query frame ``i``
+ * ([AGG] "Mask Generation"): [0, min(S, i+1)) for the retained scale frames and
+ * [max(S, i - W_f + 1), i + 1) for the window, W_f = sliding_window_size *
+ * num_frame_per_block (sliding_window_size <= 0: no window).  Touching intervals
+ * are merged.  Writes at most two [lo, hi) pairs into lo[]/hi[] and returns how
+ * many (1 or 2), or a negative status.
+ */
+int swa_sched_frame_intervals(int i, int sliding_window_size, int num_frame_per_block,
+                              int num_frame_for_scale, int* lo, int* hi);
+
+/* swa_sched_prefill: the prefill work list in launch (longest-first) order.
+ * One item = one batch row b, head h, query frame f and a pair of 128-row query
+ * tiles of that frame.  Each item is 8 int32: {b, h, f, q_row0, rows_a, rows_b,
+ * n_key_tiles, n_key_tokens}, q_row0 being the first query token of tile a
+ * within the frame's sequence (tile b starts 128 rows later; rows_b = 0 when the
+ * pair has a single tile).  Key tiles are 128-token runs of the frame's
+ * intervals; fully masked tiles never appear.  ``out`` may be NULL to query the
+ * count.  Returns the number of items (<= cap written) or a negative status. */
+int64_t swa_sched_prefill(int B, int S, int P, int heads, int sliding_window_size,
+                          int num_frame_per_block, int num_frame_for_scale,
+                          int32_t* out, int64_t cap);
+
+/* ---------------------------------------------------------------- prefill
+ * Frame-causal sliding-window attention over a whole clip ([AGG], [IO]).
+ *   q, k, v, out: [B, S*P, heads, head_dim] contiguous, i.e. the pages'
+ *                 [B*S, P, C] token layout with C = heads*head_dim.
+ *   S: number of frames, P: tokens per frame (special + patch tokens).
+ *   sliding_window_size <= 0 -> full (frame-)causal attention.
+ *   num_frame_for_scale: the first frames every later frame also sees.
+ * Query frame i attends to every token of key frame j iff j <= i and
+ * (j < num_frame_for_scale or j >= i - sliding_window_size*num_frame_per_block + 1).
+ * dtype SWA_BF16 needs head_dim 64 or 128 (tcgen05 path); SWA_F32 accepts
+ * 32, 64 or 128 (SIMT path).  Errors: SWA_ERR_ARG, SWA_ERR_SHAPE,
+ * SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA. */
+swa_status swa_prefill(const void* q, const void* k, const void* v, void* out,
+                       int B, int S, int P, int C, int heads, int head_dim,
+                       int sliding_window_size, int num_frame_per_block,
+                       int num_frame_for_scale, int dtype, void* stream);
+
+/* --------------------------------------------------------- streaming cache
+ * Per-layer rolling paged KV cache for frame-by-frame streaming ([AGG] "KV Cache
+ * Eviction Strategy"; [BLK]).  ``global_idx`` selects the layer's cache.
+ *
+ * Storage (inside the caller's device buffer): pages of ``page_tokens`` tokens.
+ * Slot s holds one frame in pages s*ppf .. s*ppf+ppf-1, ppf = ceil(P/page_tokens).
+ * Frame i < scale_frames lives in slot i; a window frame i lives in slot
+ * scale_frames + (i mod window_frames) ([SWA] slot i mod W), so the frame that
+ * arrives overwrites exactly the frame it evicts.  With cross_frame_special the
+ * evicted frame first leaves its first num_special tokens in a packed special
+ * region starting at page n_slots*ppf.  Per layer the device keeps the slot map,
+ * the page table (retained frames ascending, then special pages), the eviction of
+ * the last append and the key segments the attention kernel reads; the host keeps
+ * only a frame counter to reject out-of-order calls.
+ */
+typedef struct swa_stream_cfg {
+    int num_layers;          /* caches, indexed by global_idx in [0, num_layers)       */
+    int heads;               /* H                                                       */
+    int head_dim;            /* D                                                       */
+    int P;                   /* tokens per frame                                        */
+    int scale_frames;        /* kv_cache_scale_frames: first frames never evicted       */
+    int window_frames;       /* kv_cache_sliding_window in frames; <= 0 keeps all frames */
+    int page_tokens;         /* tokens per page (16)                                    */
+    int cross_frame_special; /* kv_cache_cross_frame_special: keep specials of evicted  */
+    int num_special;         /* camera + register tokens at the head of every frame     */
+    int max_frames;          /* frames per layer the buffer is sized for               */
+    int dtype;               /* swa_dtype of K/V/Q/out                                  */
+    int max_splits;          /* split-KV partial buffers for the attend (>= 1)          */
+} swa_stream_cfg;
+
+typedef struct swa_stream swa_stream;  /* opaque host handle */
+
+/* Device bytes swa_stream_create needs for ``cfg`` (0 if cfg is invalid). */
+size_t swa_stream_bytes(const swa_stream_cfg* cfg);
+
+/* Create a handle over ``dev_buf`` (caller-owned device memory of at least
+ * swa_stream_bytes(cfg) bytes, 256-byte aligned).  Clears the buffer on ``stream``.
+ * The handle is host memory owned by the library until swa_stream_destroy. */
+swa_status swa_stream_create(swa_stream** out, const swa_stream_cfg* cfg, void* dev_buf,
+                             size_t bytes, void* stream);
+void swa_stream_destroy(swa_stream* h);
+
+/* Empty every layer's cache (the pages' clean_kv_cache). */
+swa_status swa_stream_reset(swa_stream* h, void* stream);
+
+/* Append frame ``frame_idx`` (must equal the number of frames this layer has seen)
+ * and apply the eviction rule on the device: once more than
+ * scale_frames + window_frames full frames are cached, the oldest non-scale frame
+ * (frame_idx - window_frames) leaves -- keeping its specials if configured -- and
+ * the new frame takes its slot.  k_frame, v_frame: [P, heads, head_dim].
+ * Errors: SWA_ERR_ORDER (wrong frame index), SWA_ERR_CAPACITY (beyond max_frames
+ * or global_idx out of range). */
+swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx,
+                                   const void* k_frame, const void* v_frame, void* stream);
+
+/* The frame's queries q_frame [P, heads, head_dim] attend to everything the layer's
+ * cache holds after the append (retained full frames, the current frame and
+ * retained specials); out [P, heads, head_dim].  ``frame_idx`` must be the frame
+ * appended last (SWA_ERR_ORDER otherwise).  Uses split-KV partials in the handle's
+ * buffer: calls on one handle must not overlap on the GPU. */
+swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx,
+                             const void* q_frame, void* out, void* stream);
+
+/* Layout of one layer's metadata block, in int32 units. */
+typedef struct swa_meta_layout {
+    int n_ints;          /* size of the block                                  */
+    int n_slots;         /* slots (scale + window, or max_frames if no window) */
+    int pages_per_frame; /* ppf                                                */
+    int max_pages;       /* capacity of the page table                         */
+    int max_segs;        /* capacity of the segment list                       */
+    int off_slot_frame;  /* int32[n_slots]: frame held by each slot, -1 empty  */
+    int off_page_table;  /* int32[max_pages]: physical page ids, logical order */
+    int off_seg_row;     /* int32[max_segs]: first storage row of each segment */
+    int off_seg_len;     /* int32[max_segs]: tokens in each segment            */
+    /* header ints at offsets 0..7: n_frames, n_evicted, n_special_tokens,
+       last_evicted (-1 none), n_pages, n_segs, n_slots_used, reserved */
+} swa_meta_layout;
+
+swa_status swa_stream_meta_layout(const swa_stream* h, swa_meta_layout* out);
+
+/* Synchronous copy of layer ``global_idx``'s metadata block into host ``dst``
+ * (n_ints >= layout.n_ints).  For tests and inspection; waits for ``stream``. */
+swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, int32_t* dst,
+                               size_t n_ints, void* stream);
+
+/* Device pointers of layer ``global_idx``'s K and V page storage
+ * ([n_pages_total * page_tokens, heads, head_dim]); NULL on error. */
+void* swa_stream_k_storage(const swa_stream* h, int global_idx);
+void* swa_stream_v_storage(const swa_stream* h, int global_idx);
+
+/* ------------------------------------------------- token-band GQA prefill
+ * Mistral-style sliding-window attention ([SWA]): token t attends to s iff
+ * t - window + 1 <= s <= t; query head h reads KV head h / (Hq / Hkv).
+ *   q, out: [B, N, Hq, head_dim]; k, v: [B, N, Hkv, head_dim].
+ * bf16: head_dim 64 or 128; f32: 32, 64 or 128. */
+swa_status swa_band_prefill(const void* q, const void* k, const void* v, void* out,
+                            int B, int N, int Hq, int Hkv, int head_dim, int window,
+                            int dtype, void* stream);
+
+/* ------------------------------------------------------ rolling GQA decode
+ * One new token per sequence at position ``pos`` ([SWA]): its K/V is written into
+ * the rolling cache at slot pos mod W, then q attends over the valid slots (all W
+ * once pos >= W-1, else slots 0..pos).
+ *   q, out: [B, Hq, head_dim]; k_new, v_new: [B, Hkv, head_dim];
+ *   k_cache, v_cache: [B, W, Hkv, head_dim] (updated in place).
+ *   workspace: device scratch of at least swa_decode_workspace_bytes(...) bytes
+ *   (split-K partials); calls sharing a workspace must not overlap on the GPU.
+ * bf16: head_dim 64 or 128, Hq/Hkv <= 8; f32: 32, 64 or 128. */
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int head_dim, int W);
+swa_status swa_decode(const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, long long pos, int W,
+                      int B, int Hq, int Hkv, int head_dim, void* out,
+                      void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* ------------------------------------------------------- device errors
+ * Kernels bound every wait; a wait that runs out latches a device flag and the
+ * kernel returns early.  swa_device_error_check synchronizes ``stream``, reads and
+ * clears the flag and returns SWA_ERR_TIMEOUT if it was set (SWA_OK otherwise).
+ * swa_debug_wait_timeout launches one thread that waits on a flag nothing sets for
+ * ``timeout_us`` microseconds, so tests can exercise that path. */
+swa_status swa_device_error_check(void* stream);
+swa_status swa_debug_wait_timeout(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SWA_B200_H */

@@ -1,0 +1,286 @@
+"""Python binding of libswa_b200.so (frame-causal sliding-window attention on B200).
+
+Argument marshalling only: every function forwards tensor data pointers, sizes
+and the current CUDA stream to the C ABI of ``include/swa.h`` under the same
+name, and raises :class:`SwaError` on a non-zero status.  All arithmetic runs
+in the library's CUDA kernels; there is no fallback.  Importing this module
+fails if the library has not been built (``python -m
+streaming_frame_causal_b200.build``).
+
+Tensor layouts follow the pages' contracts: tokens [B, S*P, heads, head_dim]
+(the [B*S, P, C] layout with C = heads*head_dim), streaming frames
+[P, heads, head_dim], decode tensors [B, heads, head_dim] and caches
+[B, W, Hkv, head_dim].
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libswa_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "swa.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m streaming_frame_causal_b200.build`")
+_lib = C.CDLL(LIB_PATH)
+
+SWA_F32, SWA_BF16 = 0, 1
+STATUS = {0: "SWA_OK", -1: "SWA_ERR_ARG", -2: "SWA_ERR_SHAPE", -3: "SWA_ERR_ORDER",
+          -4: "SWA_ERR_CAPACITY", -5: "SWA_ERR_CUDA", -6: "SWA_ERR_TIMEOUT", -7: "SWA_ERR_UNSUPPORTED"}
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_lib.swa_status_str(status).decode()})")
+
+
+class swa_stream_cfg(C.Structure):
+    _fields_ = [(n, C.c_int) for n in (
+        "num_layers", "heads", "head_dim", "P", "scale_frames", "window_frames", "page_tokens",
+        "cross_frame_special", "num_special", "max_frames", "dtype", "max_splits")]
+
+
+class swa_meta_layout(C.Structure):
+    _fields_ = [(n, C.c_int) for n in (
+        "n_ints", "n_slots", "pages_per_frame", "max_pages", "max_segs", "off_slot_frame",
+        "off_page_table", "off_seg_row", "off_seg_len")]
+
+
+_vp, _i, _i64, _sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+_sigs = {
+    "swa_status_str": (C.c_char_p, [_i]),
+    "swa_version": (_i, []),
+    "swa_sched_frame_intervals": (_i, [_i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i)]),
+    "swa_sched_prefill": (_i64, [_i, _i, _i, _i, _i, _i, _i, _vp, _i64]),
+    "swa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "swa_stream_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
+    "swa_stream_create": (_i, [C.POINTER(_vp), C.POINTER(swa_stream_cfg), _vp, _sz, _vp]),
+    "swa_stream_destroy": (None, [_vp]),
+    "swa_stream_reset": (_i, [_vp, _vp]),
+    "swa_stream_append_evict": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "swa_stream_attend": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
+    "swa_stream_get_meta": (_i, [_vp, _i, _vp, _sz, _vp]),
+    "swa_stream_k_storage": (_vp, [_vp, _i]),
+    "swa_stream_v_storage": (_vp, [_vp, _i]),
+    "swa_band_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "swa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "swa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, C.c_longlong, _i, _i, _i, _i, _i, _vp, _vp, _sz,
+                        _i, _vp]),
+    "swa_device_error_check": (_i, [_vp]),
+    "swa_debug_wait_timeout": (_i, [_i, _vp]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def header_functions() -> list[str]:
+    """Names of every function include/swa.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(swa_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SwaError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SWA_BF16
+    if t.dtype == torch.float32:
+        return SWA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# --------------------------------------------------------------- scheduler
+def swa_sched_frame_intervals(i: int, sliding_window_size: int, num_frame_per_block: int,
+                              num_frame_for_scale: int) -> list[tuple[int, int]]:
+    lo = (C.c_int * 2)()
+    hi = (C.c_int * 2)()
+    n = _lib.swa_sched_frame_intervals(i, sliding_window_size, num_frame_per_block, num_frame_for_scale,
+                                       lo, hi)
+    if n < 0:
+        raise SwaError(n, "swa_sched_frame_intervals")
+    return [(lo[j], hi[j]) for j in range(n)]
+
+
+def swa_sched_prefill(B: int, S: int, P: int, heads: int, sliding_window_size: int,
+                      num_frame_per_block: int, num_frame_for_scale: int):
+    """Prefill work list as an int32 numpy array [items, 8] (see include/swa.h)."""
+    import numpy as np
+    n = _lib.swa_sched_prefill(B, S, P, heads, sliding_window_size, num_frame_per_block,
+                               num_frame_for_scale, None, 0)
+    if n < 0:
+        raise SwaError(int(n), "swa_sched_prefill")
+    out = np.zeros((n, 8), dtype=np.int32)
+    _lib.swa_sched_prefill(B, S, P, heads, sliding_window_size, num_frame_per_block, num_frame_for_scale,
+                           out.ctypes.data, n)
+    return out
+
+
+# ---------------------------------------------------------------- prefill
+def swa_prefill(q, k, v, out, S: int, P: int, sliding_window_size: int, num_frame_per_block: int = 1,
+                num_frame_for_scale: int = 0, stream=None) -> torch.Tensor:
+    """Frame-causal sliding-window attention; q/k/v/out [B, S*P, heads, head_dim]."""
+    B, N, H, D = q.shape
+    _check(_lib.swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, P, H * D, H, D,
+                            sliding_window_size, num_frame_per_block, num_frame_for_scale,
+                            _dtype_code(q), _stream(stream)), "swa_prefill")
+    return out
+
+
+def swa_band_prefill(q, k, v, out, window: int, stream=None) -> torch.Tensor:
+    """Token-band GQA attention; q/out [B, N, Hq, D], k/v [B, N, Hkv, D]."""
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _check(_lib.swa_band_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, Hq, Hkv, D, window,
+                                 _dtype_code(q), _stream(stream)), "swa_band_prefill")
+    return out
+
+
+# ----------------------------------------------------------------- decode
+def swa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, head_dim: int, W: int) -> int:
+    return int(_lib.swa_decode_workspace_bytes(B, Hq, Hkv, head_dim, W))
+
+
+def swa_decode(q, k_new, v_new, k_cache, v_cache, pos: int, out, workspace=None, stream=None):
+    """One token per sequence at ``pos``; caches [B, W, Hkv, D] are updated in place."""
+    B, Hq, D = q.shape
+    W, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if workspace is None:
+        n = swa_decode_workspace_bytes(B, Hq, Hkv, D, W)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _check(_lib.swa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), int(pos), W,
+                           B, Hq, Hkv, D, _ptr(out), _ptr(workspace), workspace.numel(),
+                           _dtype_code(q), _stream(stream)), "swa_decode")
+    return out
+
+
+# ----------------------------------------------------------------- errors
+def swa_device_error_check(stream=None) -> int:
+    """Synchronizes and returns the status of the latched device error flag (0 = none)."""
+    return int(_lib.swa_device_error_check(_stream(stream)))
+
+
+def swa_debug_wait_timeout(timeout_us: int, stream=None) -> None:
+    _check(_lib.swa_debug_wait_timeout(int(timeout_us), _stream(stream)), "swa_debug_wait_timeout")
+
+
+def swa_status_str(status: int) -> str:
+    return _lib.swa_status_str(int(status)).decode()
+
+
+def swa_version() -> int:
+    return int(_lib.swa_version())
+
+
+# -------------------------------------------------------------- streaming
+def _make_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_tokens,
+              cross_frame_special, num_special, max_frames, dtype, max_splits):
+    return swa_stream_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_tokens,
+                          int(bool(cross_frame_special)), num_special, max_frames,
+                          SWA_BF16 if dtype == torch.bfloat16 else SWA_F32, max_splits)
+
+
+def swa_stream_bytes(**cfg) -> int:
+    return int(_lib.swa_stream_bytes(C.byref(_make_cfg(**cfg))))
+
+
+class SwaStream:
+    """Rolling paged KV cache over a torch-owned device buffer (one per model)."""
+
+    def __init__(self, num_layers: int, heads: int, head_dim: int, P: int, scale_frames: int,
+                 window_frames: int, page_tokens: int = 16, cross_frame_special: bool = False,
+                 num_special: int = 5, max_frames: int = 1024, dtype=torch.bfloat16, max_splits: int = 16,
+                 device="cuda", stream=None):
+        self.cfg = _make_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_tokens,
+                             cross_frame_special, num_special, max_frames, dtype, max_splits)
+        self.nbytes = int(_lib.swa_stream_bytes(C.byref(self.cfg)))
+        if self.nbytes == 0:
+            raise SwaError(-1, "swa_stream_bytes")
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        h = C.c_void_p()
+        _check(_lib.swa_stream_create(C.byref(h), C.byref(self.cfg), self.buf.data_ptr(), self.nbytes,
+                                      _stream(stream)), "swa_stream_create")
+        self.handle = h
+        lay = swa_meta_layout()
+        _check(_lib.swa_stream_meta_layout(self.handle, C.byref(lay)), "swa_stream_meta_layout")
+        self.layout = lay
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            _lib.swa_stream_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def swa_stream_reset(self, stream=None) -> None:
+        _check(_lib.swa_stream_reset(self.handle, _stream(stream)), "swa_stream_reset")
+
+    def swa_stream_append_evict(self, global_idx: int, frame_idx: int, k_frame, v_frame, stream=None):
+        _check(_lib.swa_stream_append_evict(self.handle, global_idx, frame_idx, _ptr(k_frame),
+                                            _ptr(v_frame), _stream(stream)), "swa_stream_append_evict")
+
+    def swa_stream_attend(self, global_idx: int, frame_idx: int, q_frame, out, stream=None):
+        _check(_lib.swa_stream_attend(self.handle, global_idx, frame_idx, _ptr(q_frame), _ptr(out),
+                                      _stream(stream)), "swa_stream_attend")
+        return out
+
+    def swa_stream_get_meta(self, global_idx: int, stream=None) -> dict:
+        import numpy as np
+        lay = self.layout
+        raw = np.zeros(lay.n_ints, dtype=np.int32)
+        _check(_lib.swa_stream_get_meta(self.handle, global_idx, raw.ctypes.data, lay.n_ints,
+                                        _stream(stream)), "swa_stream_get_meta")
+        n_pages, n_segs = int(raw[4]), int(raw[5])
+        return {
+            "n_frames": int(raw[0]), "n_evicted": int(raw[1]), "n_special": int(raw[2]),
+            "last_evicted": int(raw[3]), "n_pages": n_pages, "n_segs": n_segs, "n_retained": int(raw[6]),
+            "slot_frame": raw[lay.off_slot_frame:lay.off_slot_frame + lay.n_slots].copy(),
+            "page_table": raw[lay.off_page_table:lay.off_page_table + n_pages].copy(),
+            "seg_row": raw[lay.off_seg_row:lay.off_seg_row + n_segs].copy(),
+            "seg_len": raw[lay.off_seg_len:lay.off_seg_len + n_segs].copy(),
+        }
+
+    def storage(self, global_idx: int, which: str = "k") -> torch.Tensor:
+        """View of a layer's K or V page storage as [rows, heads, head_dim]."""
+        fn = _lib.swa_stream_k_storage if which == "k" else _lib.swa_stream_v_storage
+        addr = fn(self.handle, global_idx)
+        if not addr:
+            raise SwaError(-4, "swa_stream_storage")
+        c = self.cfg
+        esize = 2 if c.dtype == SWA_BF16 else 4
+        rows = (self.layout.max_pages * c.page_tokens)
+        off = addr - self.buf.data_ptr()
+        view = self.buf[off:off + rows * c.heads * c.head_dim * esize]
+        dt = torch.bfloat16 if c.dtype == SWA_BF16 else torch.float32
+        return view.view(dt).view(rows, c.heads, c.head_dim)

@@ -1,0 +1,583 @@
+// attn_tc.cu -- tcgen05 / TMEM / TMA attention kernel for sm_100a (bf16 in,
+// f32 accumulate, bf16 out), used by the frame-causal prefill, the streaming
+// attend (split-KV with a combine pass) and the token-band GQA prefill.
+//
+// What it computes: O = softmax(Q K^T / sqrt(D)) V over the keys the schedule
+// lists for a 128-row query tile ("Sliding Window Attention Mechanism in
+// AggregatorStream", "Mask Generation in CausalAttention": only in-window
+// frames are visible; "KV Cache Eviction Strategy": only retained frames are in
+// the cache; sliding-window explainer: token band t-W+1..t).
+//
+// CTA organisation (320 threads, one CTA per SM):
+//   warp 0      TMA producer: Q tiles once, then K/V key tiles into a ring
+//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
+//   warps 2-5   softmax for query tile A (one thread per query row)
+//   warps 6-9   softmax for query tile B
+// The two query tiles ping-pong: while softmax A turns S_A into P_A, the tensor
+// core runs P_B V and Q_B K^T, and the other way round.  S (f32, 128 columns),
+// P (bf16 pairs, 64 columns) and O (f32, D columns) of each tile live in tensor
+// memory; P feeds the PV product straight from TMEM (A operand), so the only
+// shared-memory operands are Q, K and V, staged by TMA with 128-byte swizzle.
+// Online softmax uses exp2 with the scale folded in and skips rescaling O
+// unless the running maximum grows by more than 2^8 (exact after the final
+// division by the row sum).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tile_sched.h"
+
+namespace swa {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kRows = kTileRows;       // 128
+constexpr int kSubBytes = 128 * 128;   // one 128-row x 64-column bf16 sub-tile (16 KB)
+
+template <int D>
+struct Plan {
+  static_assert(D == 64, "tcgen05 path: head_dim 64 in this kernel");
+  static constexpr int kSubs = D / 64;                 // 64-column sub-tiles per row
+  static constexpr int kTileBytes = kRows * D * 2;     // Q, K or V tile
+  static constexpr int kStages = 4;                    // K/V ring depth
+  // tensor-memory columns
+  SWA_DEV static uint32_t col_s(int g) { return g ? 128u : 0u; }
+  SWA_DEV static uint32_t col_p(int g) { return g ? 320u : 256u; }
+  SWA_DEV static uint32_t col_o(int g) { return g ? 448u : 384u; }
+  static constexpr uint32_t kTmemCols = 512;
+  // shared-memory layout (offsets from a 1024-aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
+};
+
+struct Work {
+  int b, kvh;
+  int h[2];
+  int row0[2];   // first query row of each tile (row index in the Q tensor, per batch)
+  int rows[2];   // valid query rows (0 = tile absent)
+  int t_begin, t_end;
+  int split;     // >= 0: write split-KV partials; -1: write the final output
+  int nseg;
+  int lrow[2], llen[2];
+  const int* grow;
+  const int* glen;
+  SWA_DEV int seg_row(int s) const { return grow ? __ldg(grow + s) : lrow[s]; }
+  SWA_DEV int seg_len(int s) const { return glen ? __ldg(glen + s) : llen[s]; }
+};
+
+struct Cursor {
+  int s, off;
+};
+
+SWA_DEV bool cursor_seek(const Work& w, int t, Cursor& c) {
+  c.s = 0;
+  c.off = 0;
+  while (c.s < w.nseg) {
+    const int n = cdiv(w.seg_len(c.s), kRows);
+    if (t < n) {
+      c.off = t * kRows;
+      return true;
+    }
+    t -= n;
+    ++c.s;
+  }
+  return false;
+}
+
+SWA_DEV void cursor_tile(const Work& w, const Cursor& c, int* row0, int* valid) {
+  const int len = w.seg_len(c.s);
+  *row0 = w.seg_row(c.s) + c.off;
+  *valid = imin(kRows, len - c.off);
+}
+
+SWA_DEV void cursor_next(const Work& w, Cursor& c) {
+  c.off += kRows;
+  if (c.off >= w.seg_len(c.s)) {
+    ++c.s;
+    c.off = 0;
+  }
+}
+
+SWA_DEV int total_tiles(const Work& w) {
+  int T = 0;
+  for (int s = 0; s < w.nseg; ++s) T += cdiv(w.seg_len(s), kRows);
+  return T;
+}
+
+SWA_DEV Work decode_work(const TcParams& p) {
+  Work w;
+  w.grow = nullptr;
+  w.glen = nullptr;
+  w.split = -1;
+  w.nseg = 0;
+  const int64_t bid = blockIdx.x;
+  if (p.mode == TC_FRAME) {
+    const PrefillItem it = prefill_item(bid, p.B, p.Hq, p.F, p.n_pairs);
+    w.b = it.b;
+    w.kvh = it.h / (p.Hq / p.Hkv);
+    w.h[0] = w.h[1] = it.h;
+    const int t0 = 2 * it.pair;
+    w.rows[0] = qtile_rows(p.P, t0);
+    w.rows[1] = qtile_rows(p.P, t0 + 1);
+    w.row0[0] = it.f * p.P + t0 * kRows;
+    w.row0[1] = w.row0[0] + kRows;
+    int lo[2], hi[2];
+    w.nseg = frame_intervals(it.f, p.Wf, p.S, lo, hi);
+    for (int s = 0; s < w.nseg; ++s) {
+      w.lrow[s] = lo[s] * p.P;
+      w.llen[s] = (hi[s] - lo[s]) * p.P;
+    }
+    w.t_begin = 0;
+    w.t_end = total_tiles(w);
+  } else if (p.mode == TC_BAND) {
+    const BandItem it = band_item(bid, p.B, p.Hq, p.Hkv, p.n_qtiles);
+    w.b = it.b;
+    w.kvh = it.kvh;
+    const int t0 = it.t * kRows;
+    const int rows = imin(kRows, p.Nq - t0);
+    w.h[0] = it.h0;
+    w.h[1] = it.h1 < 0 ? it.h0 : it.h1;
+    w.row0[0] = w.row0[1] = t0;
+    w.rows[0] = rows;
+    w.rows[1] = it.h1 < 0 ? 0 : rows;
+    int lo, hi;
+    band_keys(t0, rows, p.W, &lo, &hi);
+    w.nseg = 1;
+    w.lrow[0] = lo;
+    w.llen[0] = hi - lo;
+    w.t_begin = 0;
+    w.t_end = total_tiles(w);
+  } else {  // TC_STREAM
+    const StreamItem it = stream_item(bid, p.Hq, p.n_pairs);
+    w.b = 0;
+    w.kvh = it.h / (p.Hq / p.Hkv);
+    w.h[0] = w.h[1] = it.h;
+    const int t0 = 2 * it.pair;
+    w.rows[0] = qtile_rows(p.P, t0);
+    w.rows[1] = qtile_rows(p.P, t0 + 1);
+    w.row0[0] = t0 * kRows;
+    w.row0[1] = w.row0[0] + kRows;
+    w.grow = p.seg_row;
+    w.glen = p.seg_len;
+    const int n = __ldg(p.meta_hdr + 5);
+    w.nseg = (n >= 0 && n <= p.max_segs) ? n : 0;
+    const int T = total_tiles(w);
+    split_range(T, p.splits, it.split, &w.t_begin, &w.t_end);
+    w.split = (p.splits > 1) ? it.split : -1;
+  }
+  return w;
+}
+
+// Masked columns of a 64-column chunk of S become -inf: the unused tail of the
+// last tile of a key run (``cut``), or outside the band t-W+1..t.
+SWA_DEV void mask_cols(uint32_t* x, int c0, bool cut, bool band_edge, int kvalid, int krow, int qrow, int W) {
+  if (cut) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+      if (c0 + c >= kvalid) x[c] = __float_as_uint(-INFINITY);
+  } else if (band_edge) {
+    const int lo = qrow - W + 1;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const int key = krow + c0 + c;
+      if (c0 + c >= kvalid || key < lo || key > qrow) x[c] = __float_as_uint(-INFINITY);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
+  using PL = Plan<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw_base);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const Work w = decode_work(p);
+  const int T = w.t_end - w.t_begin;
+  const bool has_b = w.rows[1] > 0;
+
+  // barriers
+  const uint32_t bar0 = base + PL::kOffBar;
+  auto q_full = [&](int g) { return bar0 + 8u * g; };
+  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + PL::kStages + s); };
+  auto s_full = [&](int g) { return bar0 + 8u * (2 + 2 * PL::kStages + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (4 + 2 * PL::kStages + g); };
+  const uint32_t o_full = bar0 + 8u * (6 + 2 * PL::kStages);
+  const uint32_t drain = bar0 + 8u * (7 + 2 * PL::kStages);
+  const uint32_t tmem_slot = base + PL::kOffTmem;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full(0), 1);
+    mbar_init(q_full(1), 1);
+    for (int s = 0; s < PL::kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(s_full(0), 1);
+    mbar_init(s_full(1), 1);
+    mbar_init(p_full(0), 128);
+    mbar_init(p_full(1), 128);
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, PL::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + PL::kOffTmem);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      for (int g = 0; g < (has_b ? 2 : 1); ++g) {
+        mbar_arrive_expect_tx(q_full(g), PL::kTileBytes);
+        for (int sub = 0; sub < PL::kSubs; ++sub)
+          tma_load_4d(base + PL::kOffQ + g * PL::kTileBytes + sub * kSubBytes, &p.tm_q, q_full(g),
+                      sub * 64, w.h[g], w.row0[g], w.b);
+      }
+      Cursor cur;
+      bool ok = cursor_seek(w, w.t_begin, cur);
+      if (!ok) atomicOr(p.err, ERR_BAD_META);
+      int issued = 0;
+      for (int j = 0; j < T && ok; ++j) {
+        const int st = j % PL::kStages;
+        if (j >= PL::kStages &&
+            !mbar_wait(kv_empty(st), ((j / PL::kStages) - 1) & 1, p.err, ERR_WAIT_TMA)) {
+          ok = false;
+          break;
+        }
+        if (cur.s >= w.nseg) {
+          atomicOr(p.err, ERR_BAD_META);
+          ok = false;
+          break;
+        }
+        int krow, kvalid;
+        cursor_tile(w, cur, &krow, &kvalid);
+        mbar_arrive_expect_tx(kv_full(st), 2 * PL::kTileBytes);
+        for (int sub = 0; sub < PL::kSubs; ++sub) {
+          tma_load_4d(base + PL::kOffK + st * PL::kTileBytes + sub * kSubBytes, &p.tm_k,
+                      kv_full(st), sub * 64, w.kvh, krow, w.b);
+          tma_load_4d(base + PL::kOffV + st * PL::kTileBytes + sub * kSubBytes, &p.tm_v,
+                      kv_full(st), sub * 64, w.kvh, krow, w.b);
+        }
+        cursor_next(w, cur);
+        ++issued;
+      }
+      // drain: never leave the CTA with a bulk copy still writing its shared memory
+      for (int j = issued - PL::kStages; j < issued; ++j) {
+        if (j < 0) continue;
+        mbar_wait(kv_full(j % PL::kStages), (j / PL::kStages) & 1, p.err, ERR_WAIT_TMA);
+      }
+      for (int g = 0; g < (has_b ? 2 : 1); ++g) mbar_wait(q_full(g), 0, p.err, ERR_WAIT_TMA);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
+      auto issue_qk = [&](int g, int st) {
+        const uint32_t qa = base + PL::kOffQ + g * PL::kTileBytes;
+        const uint32_t kb = base + PL::kOffK + st * PL::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+          mma_ss(tmem + PL::col_s(g), sdesc_sw128(qa + off, 16, 1024),
+                 sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int g, int st, bool acc) {
+        const uint32_t vb = base + PL::kOffV + st * PL::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          mma_ts(tmem + PL::col_o(g), tmem + PL::col_p(g) + kk * 8,
+                 sdesc_sw128(vb + kk * 16 * 128, kSubBytes, 1024), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full(0), 0, p.err, ERR_WAIT_MMA);
+      if (ok && has_b) ok = mbar_wait(q_full(1), 0, p.err, ERR_WAIT_MMA);
+      if (ok) ok = mbar_wait(kv_full(0), 0, p.err, ERR_WAIT_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(s_full(0));
+        if (has_b) {
+          issue_qk(1, 0);
+          mma_commit(s_full(1));
+        }
+      }
+      for (int j = 0; j < T && ok; ++j) {
+        const int st = j % PL::kStages;
+        const int st1 = (j + 1) % PL::kStages;
+        const bool more = j + 1 < T;
+        if (!mbar_wait(p_full(0), j & 1, p.err, ERR_WAIT_MMA)) break;
+        tc_fence_after();
+        issue_pv(0, st, j > 0);
+        if (more) {
+          if (!mbar_wait(kv_full(st1), ((j + 1) / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+          mma_commit(s_full(0));
+        }
+        if (has_b) {
+          if (!mbar_wait(p_full(1), j & 1, p.err, ERR_WAIT_MMA)) break;
+          tc_fence_after();
+          issue_pv(1, st, j > 0);
+        }
+        mma_commit(kv_empty(st));
+        if (has_b && more) {
+          issue_qk(1, st1);
+          mma_commit(s_full(1));
+        }
+        if (!more) mma_commit(o_full);
+      }
+      // drain every MMA this thread issued before the CTA may free TMEM
+      mma_commit(drain);
+      mbar_wait(drain, 0, p.err, ERR_WAIT_MMA);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int g = (warp - 2) >> 2;  // 0: tile A, 1: tile B
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + PL::col_s(g);
+    const uint32_t tP = tmem + lane_off + PL::col_p(g);
+    const uint32_t tO = tmem + lane_off + PL::col_o(g);
+    const float sl2 = p.scale_log2;
+    const bool band = (p.mode == TC_BAND);
+    const int qrow = w.row0[g] + r;  // query token (band mode: absolute position)
+    float m = -INFINITY;             // running max of raw scores
+    float l = 0.f;                   // running row sum (relative to m)
+    bool ok = (g == 0 || has_b) && T > 0;
+    const bool active = ok;
+    Cursor cur;
+    if (ok) ok = cursor_seek(w, w.t_begin, cur);
+    for (int j = 0; j < T && ok; ++j) {
+      if (cur.s >= w.nseg) {
+        ok = false;
+        break;
+      }
+      int krow, kvalid;
+      cursor_tile(w, cur, &krow, &kvalid);
+      cursor_next(w, cur);
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), j & 1, p.err, ERR_WAIT_SOFTMAX))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // ---- pass 1: row max over the tile (masked columns excluded)
+      const bool band_edge =
+          band && !((krow >= w.row0[g] + w.rows[g] - 1 - p.W + 1) && (krow + kvalid - 1 <= w.row0[g]) &&
+                    kvalid == kRows);
+      const bool cut = !band && kvalid < kRows;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t x[64];
+        tmem_ld32(tS + c0, x);
+        tmem_ld32(tS + c0 + 32, x + 32);
+        tmem_wait_ld();
+        mask_cols(x, c0, cut, band_edge, kvalid, krow, qrow, p.W);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          mx0 = fmaxf(mx0, __uint_as_float(x[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(x[c + 1]));
+        }
+      }
+      const float tmax = fmaxf(mx0, mx1);
+      const float m_new = fmaxf(m, tmax);
+      const bool grow = (m != -INFINITY) && ((m_new - m) * sl2 > 8.0f);
+      float alpha = 1.f;
+      if (m == -INFINITY) {
+        m = m_new;
+      } else if (grow) {
+        alpha = ex2_approx((m - m_new) * sl2);
+        m = m_new;
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+        // O of this tile is complete up to key tile j-1 (the commit that
+        // signalled S_j covers the earlier PV), so it can be rescaled in place
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c0, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+          tmem_st32(tO + c0, orr);
+        }
+        tmem_wait_st();
+      }
+      l *= alpha;
+      // ---- pass 2: P = 2^(s*scale - m*scale) as bf16 pairs into TMEM
+      const float nb = (m == -INFINITY) ? 0.f : -m * sl2;
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t x[64];
+        tmem_ld32(tS + c0, x);
+        tmem_ld32(tS + c0 + 32, x + 32);
+        tmem_wait_ld();
+        mask_cols(x, c0, cut, band_edge, kvalid, krow, qrow, p.W);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(x[c]), sl2, nb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(x[c + 1]), sl2, nb));
+          sum0 += p0;
+          sum1 += p1;
+          x[c >> 1] = pack_bf16x2(p0, p1);  // index c/2 <= c: already consumed
+        }
+        tmem_st32(tP + (c0 >> 1), x);
+      }
+      l += sum0 + sum1;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(g));
+    }
+    // ---- epilogue
+    if (active && ok) {
+      if (__all_sync(0xffffffffu, mbar_wait(o_full, 0, p.err, ERR_WAIT_EPI))) {
+        tc_fence_after();
+        uint32_t orr[D];
+#pragma unroll
+        for (int c = 0; c < D; c += 32) tmem_ld32(tO + c, orr + c);
+        tmem_wait_ld();
+        if (r < w.rows[g]) {
+          const int row = w.row0[g] + r;
+          if (w.split < 0) {
+            const float inv = 1.f / l;
+            __nv_bfloat16* dst =
+                reinterpret_cast<__nv_bfloat16*>(p.out) + ((static_cast<int64_t>(w.b) * p.Nq + row) * p.Hq + w.h[g]) * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(orr[c + 0]) * inv, __uint_as_float(orr[c + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(orr[c + 2]) * inv, __uint_as_float(orr[c + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(orr[c + 4]) * inv, __uint_as_float(orr[c + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(orr[c + 6]) * inv, __uint_as_float(orr[c + 7]) * inv);
+              *reinterpret_cast<uint4*>(dst + c) = v;
+            }
+          } else {
+            const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
+            float* dst = p.part_o + idx * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 4) {
+              float4 v = make_float4(__uint_as_float(orr[c]), __uint_as_float(orr[c + 1]),
+                                     __uint_as_float(orr[c + 2]), __uint_as_float(orr[c + 3]));
+              *reinterpret_cast<float4*>(dst + c) = v;
+            }
+            p.part_ml[idx * 2 + 0] = m * sl2;
+            p.part_ml[idx * 2 + 1] = l;
+          }
+        }
+      }
+    } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < w.rows[g]) {
+      // empty split: contributes nothing to the combine
+      const int row = w.row0[g] + r;
+      const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
+      p.part_ml[idx * 2 + 0] = -INFINITY;
+      p.part_ml[idx * 2 + 1] = 0.f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, PL::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c  (m in log2 units), the
+// log-sum-exp merge of split-KV partials.  One warp per (row, head).
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part_o,
+                                                      const float* __restrict__ part_ml,
+                                                      __nv_bfloat16* __restrict__ out, int rows,
+                                                      int H, int splits) {
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows * H) return;
+  const int64_t stride = static_cast<int64_t>(rows) * H;
+  float M = -INFINITY;
+  for (int c = 0; c < splits; ++c) M = fmaxf(M, part_ml[(c * stride + gw) * 2]);
+  constexpr int E = D / 32;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float L = 0.f;
+  for (int c = 0; c < splits; ++c) {
+    const float mc = part_ml[(c * stride + gw) * 2];
+    if (mc == -INFINITY) continue;
+    const float wgt = exp2f(mc - M);
+    L += wgt * part_ml[(c * stride + gw) * 2 + 1];
+    const float* src = part_o + (c * stride + gw) * D;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] += wgt * src[lane + 32 * e];
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int e = 0; e < E; ++e) out[static_cast<int64_t>(gw) * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+}
+
+}  // namespace
+
+int tc_smem_bytes(int head_dim) {
+  return head_dim == 64 ? Plan<64>::kSmemBytes : -1;
+}
+
+cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream) {
+  if (head_dim != 64) return cudaErrorInvalidValue;
+  if (n_items <= 0) return cudaSuccess;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Plan<64>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  attn_tc_kernel<64><<<static_cast<unsigned>(n_items), kThreads, Plan<64>::kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
+                           int head_dim, int splits, cudaStream_t stream) {
+  const int warps = rows * H;
+  const int blocks = (warps + 7) / 8;
+  if (blocks == 0) return cudaSuccess;
+  auto* o = reinterpret_cast<__nv_bfloat16*>(out);
+  if (head_dim == 64)
+    combine_kernel<64><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits);
+  else if (head_dim == 128)
+    combine_kernel<128><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace swa

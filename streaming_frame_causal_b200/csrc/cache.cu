@@ -1,0 +1,148 @@
+// cache.cu -- device-side append + eviction for the rolling paged KV cache.
+//
+// Rule ("Sliding Window Attention Mechanism in AggregatorStream", section "KV
+// Cache Eviction Strategy"): after frame i is appended, when more than
+// window + scale frames are cached, cache positions [scale, n - window) leave,
+// i.e. the single oldest non-scale frame i - window.  With
+// kv_cache_cross_frame_special (same page, FAQ "Can special tokens persist
+// outside the sliding window?") that frame's leading special tokens (camera,
+// registers) move to a packed special region first.  Frame i lives in slot i
+// (scale frame) or scale + (i mod window) -- the rolling-buffer rule "slot i
+// modulo W" of the sliding-window explainer, applied to frames -- so the new
+// frame lands exactly on the slot it frees.  Eviction happens before the
+// attention kernel runs (same page: evict before attention).
+//
+// One launch does everything: each 16-byte chunk of the new frame is copied by
+// one thread; the thread whose chunk overlaps the evicted frame's special
+// tokens first moves the old chunk to the special region, so nothing races.
+// Block 0 rewrites the layer's metadata (slot map, page table, key segments,
+// counters) -- all pure functions of the frame index.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tile_sched.h"
+
+namespace swa {
+namespace {
+
+__global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p) {
+  const int i = p.frame;
+  const int slot = stream_slot(i, p.S, p.Wc);
+  const int ev = stream_evicted(i, p.S, p.Wc);
+  const int chunks = p.row_bytes >> 4;
+  const int64_t per_tensor = static_cast<int64_t>(p.P) * chunks;
+  const int64_t slot_row0 = static_cast<int64_t>(slot) * p.ppf * p.page_tokens;
+  const int64_t special_row0 = static_cast<int64_t>(p.n_slots) * p.ppf * p.page_tokens;
+  const bool move_special = (ev >= 0) && p.cross_special;
+
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < 2 * per_tensor;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int tsel = static_cast<int>(idx / per_tensor);
+    const int64_t rem = idx - tsel * per_tensor;
+    const int row = static_cast<int>(rem / chunks);
+    const int ch = static_cast<int>(rem - static_cast<int64_t>(row) * chunks);
+    uint8_t* store = tsel ? p.v_store : p.k_store;
+    const uint8_t* src = tsel ? p.v_src : p.k_src;
+    uint4* dst = reinterpret_cast<uint4*>(store + (slot_row0 + row) * p.row_bytes) + ch;
+    if (move_special && row < p.num_special) {
+      const int64_t sp_row = special_row0 + static_cast<int64_t>(ev - p.S) * p.num_special + row;
+      reinterpret_cast<uint4*>(store + sp_row * p.row_bytes)[ch] = *dst;
+    }
+    *dst = reinterpret_cast<const uint4*>(src + static_cast<int64_t>(row) * p.row_bytes)[ch];
+  }
+
+  if (blockIdx.x != 0) return;
+  // ---------------------------------------------------------------- metadata
+  int* hdr = p.meta;
+  int* slot_frame = p.meta + p.off_slot_frame;
+  int* pages = p.meta + p.off_page_table;
+  int* seg_row = p.meta + p.off_seg_row;
+  int* seg_len = p.meta + p.off_seg_len;
+  const int n_scale = imin(p.S, i + 1);
+  const int wlo = stream_window_lo(i, p.S, p.Wc);
+  const int n_ret = stream_retained(i, p.S, p.Wc);
+  const int n_ev = stream_n_evicted(i, p.S, p.Wc);
+  const int n_special = p.cross_special ? n_ev * p.num_special : 0;
+  const int sp_pages = cdiv(n_special, p.page_tokens);
+  const int n_pages = n_ret * p.ppf + sp_pages;
+  const int n_segs = n_ret + (n_special > 0 ? 1 : 0);
+  if (n_pages > p.max_pages || n_segs > p.max_segs) {
+    if (threadIdx.x == 0) atomicOr(p.err, ERR_BAD_META);
+    return;
+  }
+  // retained frame with ordinal o (ascending frame index)
+  auto ret_frame = [&](int o) { return o < n_scale ? o : wlo + (o - n_scale); };
+  for (int e = threadIdx.x; e < n_ret * p.ppf; e += blockDim.x) {
+    const int o = e / p.ppf;
+    const int pg = e - o * p.ppf;
+    pages[e] = stream_slot(ret_frame(o), p.S, p.Wc) * p.ppf + pg;
+  }
+  for (int e = threadIdx.x; e < sp_pages; e += blockDim.x) pages[n_ret * p.ppf + e] = p.n_slots * p.ppf + e;
+  for (int o = threadIdx.x; o < n_ret; o += blockDim.x) {
+    seg_row[o] = stream_slot(ret_frame(o), p.S, p.Wc) * p.ppf * p.page_tokens;
+    seg_len[o] = p.P;
+  }
+  if (threadIdx.x == 0 && n_special > 0) {
+    seg_row[n_ret] = p.n_slots * p.ppf * p.page_tokens;
+    seg_len[n_ret] = n_special;
+  }
+  // slot map: which frame each slot holds after this append
+  for (int s = threadIdx.x; s < p.n_slots; s += blockDim.x) {
+    int f = -1;
+    if (p.Wc <= 0 || s < p.S) {
+      f = (s <= i) ? s : -1;
+    } else {
+      const int r = s - p.S;  // residue of frames mapped here
+      if (i >= r) {
+        const int j = i - ((i - r) % p.Wc);  // latest frame <= i with j mod Wc == r
+        f = (j >= wlo && j >= p.S) ? j : -1;
+      }
+    }
+    slot_frame[s] = f;
+  }
+  if (threadIdx.x == 0) {
+    hdr[0] = i + 1;
+    hdr[1] = n_ev;
+    hdr[2] = n_special;
+    hdr[3] = ev;
+    hdr[4] = n_pages;
+    hdr[5] = n_segs;
+    hdr[6] = n_ret;
+    hdr[7] = 0;
+  }
+}
+
+__global__ void debug_wait_kernel(int* err, long long timeout_ns) {
+  // waits on a flag that nothing sets; gives up after timeout_ns and latches
+  // the error -- the same bounded-wait contract every kernel follows
+  __shared__ int flag;
+  flag = 0;
+  __syncthreads();
+  const uint64_t t0 = global_timer_ns();
+  while (*reinterpret_cast<volatile int*>(&flag) == 0) {
+    if (global_timer_ns() - t0 > static_cast<uint64_t>(timeout_ns)) {
+      atomicOr(err, ERR_WAIT_DEBUG);
+      return;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
+  const int64_t work = 2LL * p.P * (p.row_bytes >> 4);
+  int64_t blocks = (work + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 4096) blocks = 4096;
+  append_evict_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream) {
+  debug_wait_kernel<<<1, 1, 0, stream>>>(err, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace swa

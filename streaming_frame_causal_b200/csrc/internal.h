@@ -1,0 +1,102 @@
+// internal.h -- declarations shared by the host API (api.cu) and the kernel
+// translation units.  Not part of the public C ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace swa {
+
+enum TcMode : int { TC_FRAME = 0, TC_STREAM = 1, TC_BAND = 2 };
+
+// Parameters of the tcgen05 attention kernel (passed by value as a
+// __grid_constant__ so the TMA descriptors are addressable by the kernel).
+struct TcParams {
+  CUtensorMap tm_q;   // Q as 4-D {D, Hq, Nq, B}, box {64, 1, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_k;   // K as 4-D {D, Hkv, Nk, B}
+  CUtensorMap tm_v;   // V, same shape as K
+  void* out;          // bf16 [B, Nq, Hq, D] (final output)
+  float* part_o;      // f32 [splits, Nq, Hq, D] (split-KV partial numerators)
+  float* part_ml;     // f32 [splits, Nq, Hq, 2] (running max in log2 units, row sum)
+  const int* seg_row; // stream mode: key segments (storage row, length) on the device
+  const int* seg_len;
+  const int* meta_hdr;
+  int* err;           // device error flag
+  int mode;
+  int B, Nq, Hq, Hkv;
+  int P, F, S, Wf, n_pairs;  // frame mode (P, n_pairs also stream mode)
+  int W, n_qtiles;           // band mode
+  int splits, max_segs;      // stream mode
+  float scale_log2;          // log2(e) / sqrt(D)
+};
+
+cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream);
+int tc_smem_bytes(int head_dim);
+cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
+                           int head_dim, int splits, cudaStream_t stream);
+
+// ---------------------------------------------------------------- SIMT f32 path
+enum SimtMode : int { SIMT_FRAME = 0, SIMT_BAND = 1, SIMT_STREAM = 2, SIMT_DECODE = 3 };
+
+struct SimtParams {
+  const float* q;    // [B, Nq, Hq, D]
+  const float* k;    // [B, Nk, Hkv, D] (stream: page storage rows; decode: [B, W, Hkv, D])
+  const float* v;
+  float* out;        // [B, Nq, Hq, D]
+  const int* seg_row;
+  const int* seg_len;
+  const int* meta_hdr;
+  int* err;
+  int mode;
+  int B, Nq, Nk, Hq, Hkv, D;
+  int P, S, Wf;      // frame
+  int W;             // band
+  int n_valid;       // decode: valid slots
+  int max_segs;
+  float scale;
+};
+
+cudaError_t launch_attn_simt(const SimtParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- stream cache
+struct AppendParams {
+  const uint8_t* k_src;  // [P, H, D] of the new frame
+  const uint8_t* v_src;
+  uint8_t* k_store;      // page storage [total_rows, H, D]
+  uint8_t* v_store;
+  int* meta;             // the layer's metadata block
+  int* err;              // device error flag
+  int frame;             // index of the frame being appended
+  int P, S, Wc, ppf, page_tokens, n_slots, num_special, cross_special;
+  int row_bytes;         // H * D * element size (multiple of 16)
+  int off_slot_frame, off_page_table, off_seg_row, off_seg_len;
+  int max_pages, max_segs;
+};
+
+cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+  const void* q;      // [B, Hq, D]
+  const void* k_new;  // [B, Hkv, D]
+  const void* v_new;
+  void* k_cache;      // [B, W, Hkv, D]
+  void* v_cache;
+  void* out;          // [B, Hq, D]
+  float* part_o;      // [B, Hkv, chunks, G, D]
+  float* part_ml;     // [B, Hkv, chunks, G, 2]
+  int* err;
+  long long pos;
+  int W, B, Hq, Hkv, D, chunks, chunk_len, n_valid, slot;
+  float scale_log2;
+};
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
+int decode_chunks(int B, int Hkv, int W);
+cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- misc
+cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream);
+
+}  // namespace swa

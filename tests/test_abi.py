@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function the header declares, rejects bad arguments before touching the GPU,
+and its tile scheduler covers exactly the oracle's visible set."""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from oracle import attention as orc
+
+
+@pytest.fixture(scope="module")
+def swa():
+    from streaming_frame_causal_b200.build import build
+    build()
+    import streaming_frame_causal_b200 as m
+    return m
+
+
+def test_every_header_function_is_exported(swa):
+    names = swa.header_functions()
+    assert len(names) >= 20
+    lib = C.CDLL(swa.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(swa):
+    assert swa.swa_status_str(0) == "ok"
+    assert swa.swa_status_str(-3) == "frame out of order"
+    assert swa.swa_version() >= 100
+
+
+def _visible_from_intervals(swa, i, sws, nfpb, S):
+    out = []
+    for lo, hi in swa.swa_sched_frame_intervals(i, sws, nfpb, S):
+        out.extend(range(lo, hi))
+    return out
+
+
+@pytest.mark.parametrize("sws,nfpb,S", [(3, 1, 2), (6, 1, 8), (-1, 1, 0), (1, 1, 0), (2, 2, 1),
+                                        (4, 1, 0), (1, 1, 5), (100, 1, 3), (0, 1, 2)])
+def test_intervals_equal_oracle_visible_set(swa, sws, nfpb, S):
+    for i in range(40):
+        ivs = swa.swa_sched_frame_intervals(i, sws, nfpb, S)
+        assert 1 <= len(ivs) <= 2
+        # disjoint, ascending, not touching (touching runs are merged)
+        for (a, b), (c, d) in zip(ivs, ivs[1:]):
+            assert b < c
+        got = _visible_from_intervals(swa, i, sws, nfpb, S)
+        want = [j for j in range(i + 1) if orc.frame_visible(i, j, S, sws, nfpb)]
+        assert got == want, (i, got, want)
+
+
+@pytest.mark.parametrize("F,P,H,sws,S", [(32, 1004, 16, 6, 8), (8, 21, 2, 3, 2), (5, 128, 1, 2, 0),
+                                         (7, 129, 3, -1, 1), (3, 300, 2, 1, 0)])
+def test_prefill_schedule_covers_visible_pairs_once(swa, F, P, H, sws, S):
+    B = 2
+    items = swa.swa_sched_prefill(B, F, P, H, sws, 1, S)
+    n_pairs = -(-(-(-P // 128)) // 2)
+    assert len(items) == F * B * H * n_pairs
+    # longest first (non-increasing key tiles), nothing empty
+    assert np.all(np.diff(items[:, 6]) <= 0)
+    assert np.all(items[:, 6] > 0)
+    seen = {}
+    for b, h, f, row0, ra, rb, tiles, toks in items:
+        vis = [j for j in range(F) if orc.frame_visible(f, j, S, sws, 1)]
+        assert toks == len(vis) * P
+        # one tile per started 128 keys of each visible run, never a fully masked tile
+        runs = swa.swa_sched_frame_intervals(int(f), sws, 1, S)
+        assert tiles == sum(-(-((hi - lo) * P) // 128) for lo, hi in runs)
+        assert tiles * 128 - toks < 128 * len(runs)
+        t0 = (row0 - f * P) // 128
+        for t, rows in ((t0, ra), (t0 + 1, rb)):
+            if rows:
+                key = (b, h, f, t)
+                assert key not in seen
+                seen[key] = rows
+    # every query row of every (b, h, frame) is in exactly one tile
+    for b in range(B):
+        for h in range(H):
+            for f in range(F):
+                rows = sum(seen.get((b, h, f, t), 0) for t in range(-(-P // 128)))
+                assert rows == P
+
+
+def test_prefill_rejects_bad_shapes_before_launch(swa):
+    lib = swa._lib
+    # C != heads * head_dim
+    assert lib.swa_prefill(16, 16, 16, 16, 1, 2, 4, 100, 2, 64, 2, 1, 0, 1, None) == -2
+    # null pointers
+    assert lib.swa_prefill(None, None, None, None, 1, 2, 4, 128, 2, 64, 2, 1, 0, 1, None) == -1
+    # bad dtype
+    assert lib.swa_prefill(16, 16, 16, 16, 1, 2, 4, 128, 2, 64, 2, 1, 0, 7, None) == -1
+    # empty input is a no-op
+    assert lib.swa_prefill(None, None, None, None, 1, 0, 4, 128, 2, 64, 2, 1, 0, 1, None) == 0
+    # band: Hq not a multiple of Hkv
+    assert lib.swa_band_prefill(16, 16, 16, 16, 1, 64, 6, 4, 64, 16, 1, None) == -2
+    # decode: negative position
+    assert lib.swa_decode(16, 16, 16, 16, 16, -1, 8, 1, 4, 2, 64, 16, None, 0, 1, None) == -1
+
+
+def test_stream_geometry_sizes(swa):
+    # 8 scale + 64 window frames of 1004 tokens, 16 heads x 64, bf16: 72 slots x 63 pages
+    n = swa.swa_stream_bytes(num_layers=1, heads=16, head_dim=64, P=1004, scale_frames=8,
+                             window_frames=64, page_tokens=16, cross_frame_special=False, num_special=5,
+                             max_frames=300, dtype=__import__("torch").bfloat16, max_splits=16)
+    rows = 72 * 63 * 16
+    assert n >= 2 * rows * 16 * 64 * 2
+    n2 = swa.swa_stream_bytes(num_layers=1, heads=16, head_dim=64, P=1004, scale_frames=8,
+                              window_frames=64, page_tokens=16, cross_frame_special=True, num_special=5,
+                              max_frames=1000, dtype=__import__("torch").bfloat16, max_splits=16)
+    # special region: 928 evicted frames x 5 tokens = 4640 tokens = 290 pages
+    assert n2 - n >= 2 * 290 * 16 * 16 * 64 * 2
+    bad = swa._make_cfg(1, 16, 64, 1004, 8, 64, 16, False, 2000, 300, __import__("torch").bfloat16, 16)
+    assert swa._lib.swa_stream_bytes(C.byref(bad)) == 0

@@ -1,0 +1,149 @@
+"""Streaming rolling paged cache on the GPU: bookkeeping bit-exact against the
+oracle's host model, stored K/V bit-exact, attention outputs within tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as orc
+from tol import check_bf16, check_f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def swa():
+    import streaming_frame_causal_b200 as m
+    return m
+
+
+def _compare_meta(meta, oc, layer, i):
+    assert meta["n_frames"] == i + 1
+    assert meta["last_evicted"] == oc.layers[layer].last_evicted, i
+    assert meta["n_evicted"] == oc.layers[layer].n_evicted
+    assert meta["n_special"] == oc.n_special_tokens(layer)
+    np.testing.assert_array_equal(meta["slot_frame"], oc.slot_frames(layer))
+    np.testing.assert_array_equal(meta["page_table"], oc.page_table(layer))
+
+
+def _stream(swa, F, P, H, D, S, Wc, special, dtype, frames_to_check, max_frames=None, layers=1,
+            check_rows=None):
+    max_frames = max_frames or F
+    dev = "cuda"
+    cache = swa.SwaStream(num_layers=layers, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
+                          cross_frame_special=special, num_special=5, max_frames=max_frames, dtype=dtype)
+    oc = orc.StreamCache(heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, page_tokens=16,
+                         cross_frame_special=special, num_special=5, max_frames=max_frames, num_layers=layers)
+    for i in range(F):
+        for layer in range(layers):
+            q, k, v = synth.stream_frame(i, P=P, H=H, D=D, dtype=dtype, base_seed=layer)
+            cache.swa_stream_append_evict(layer, i, k.to(dev), v.to(dev))
+            oc.append_evict(layer, i, k.float().numpy(), v.float().numpy())
+            _compare_meta(cache.swa_stream_get_meta(layer), oc, layer, i)
+            if i in frames_to_check:
+                out = torch.empty(q.shape, dtype=dtype, device=dev)
+                cache.swa_stream_attend(layer, i, q.to(dev), out)
+                torch.cuda.synchronize()
+                got = out.float().cpu().numpy()
+                if check_rows is None:
+                    ref = oc.attend(layer, q.float().numpy())
+                else:
+                    kc, vc = oc.gather(layer)
+                    qq = q.float().numpy()[check_rows]
+                    ref = np.stack([orc.softmax_attention(qq[:, h], kc[:, h], vc[:, h]) for h in range(H)], 1)
+                    got = got[check_rows]
+                if dtype == torch.float32:
+                    check_f32(got, ref, f"frame {i}")
+                else:
+                    check_bf16(got, ref, f"frame {i}")
+    assert swa.swa_device_error_check() == 0
+    return cache, oc
+
+
+def test_tiny_config_stream_equals_prefill(swa):
+    """8 frames x 21 tokens, 2 x 32, f32: streaming through a 2+3-frame rolling
+    cache matches the oracle's prefill with window 3 and 2 scale frames."""
+    F, P, H, D = 8, 21, 2, 32
+    q, k, v = synth.tiny_qkv(seed=0)
+    full = orc.prefill(q.numpy(), k.numpy(), v.numpy(), P=P, scale_frames=2, sliding_window_size=3)[0]
+    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=2, window_frames=3,
+                          max_frames=F, dtype=torch.float32)
+    gpu_prefill = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    swa.swa_prefill(q.cuda(), k.cuda(), v.cuda(), gpu_prefill, S=F, P=P, sliding_window_size=3,
+                    num_frame_for_scale=2)
+    for i in range(F):
+        sl = slice(i * P, (i + 1) * P)
+        cache.swa_stream_append_evict(0, i, k[0, sl].contiguous().cuda(), v[0, sl].contiguous().cuda())
+        out = torch.empty(P, H, D, device="cuda")
+        cache.swa_stream_attend(0, i, q[0, sl].contiguous().cuda(), out)
+        torch.cuda.synchronize()
+        check_f32(out.cpu().numpy(), full[sl], f"stream frame {i}")
+        check_f32(out.cpu().numpy(), gpu_prefill[0, sl].cpu().numpy(), f"stream vs prefill {i}")
+
+
+@pytest.mark.parametrize("special", [False, True])
+def test_bf16_small_stream(swa, special):
+    _stream(swa, F=12, P=300, H=2, D=64, S=2, Wc=3, special=special, dtype=torch.bfloat16,
+            frames_to_check=set(range(12)))
+
+
+def test_two_layers_are_independent(swa):
+    _stream(swa, F=7, P=130, H=2, D=64, S=1, Wc=2, special=True, dtype=torch.bfloat16,
+            frames_to_check={0, 3, 6}, layers=2)
+
+
+def test_stored_pages_bit_exact(swa):
+    F, P, H, D, S, Wc = 9, 40, 2, 64, 2, 3
+    cache, oc = _stream(swa, F=F, P=P, H=H, D=D, S=S, Wc=Wc, special=True, dtype=torch.bfloat16,
+                        frames_to_check=set())
+    kst = cache.storage(0, "k").cpu()
+    ppf = -(-P // 16)
+    for j in sorted(oc.layers[0].frames):
+        s = oc.slot_of(j)
+        _, k, _ = synth.stream_frame(j, P=P, H=H, D=D)
+        assert torch.equal(kst[s * ppf * 16: s * ppf * 16 + P], k)
+    for e, j in enumerate(oc.layers[0].special_from):
+        _, k, _ = synth.stream_frame(j, P=P, H=H, D=D)
+        for r in range(5):
+            page, off = oc.special_location(e * 5 + r)
+            assert torch.equal(kst[page * 16 + off], k[r])
+
+
+def test_out_of_order_and_bounds(swa):
+    cache = swa.SwaStream(num_layers=2, heads=2, head_dim=64, P=20, scale_frames=1, window_frames=2,
+                          max_frames=4)
+    q, k, v = synth.stream_frame(0, P=20, H=2, D=64)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(q)
+    with pytest.raises(swa.SwaError) as e:
+        cache.swa_stream_attend(0, 0, q, out)          # attend before append
+    assert e.value.status == -3
+    with pytest.raises(swa.SwaError) as e:
+        cache.swa_stream_append_evict(0, 1, k, v)      # skips frame 0
+    assert e.value.status == -3
+    with pytest.raises(swa.SwaError) as e:
+        cache.swa_stream_append_evict(2, 0, k, v)      # no such layer
+    assert e.value.status == -4
+    for i in range(4):
+        cache.swa_stream_append_evict(0, i, k, v)
+    with pytest.raises(swa.SwaError) as e:
+        cache.swa_stream_append_evict(0, 4, k, v)      # beyond max_frames
+    assert e.value.status == -4
+    cache.swa_stream_reset()
+    cache.swa_stream_append_evict(0, 0, k, v)
+    assert cache.swa_stream_get_meta(0)["n_frames"] == 1
+
+
+def test_300_frame_stream(swa):
+    """8 scale + 64 window frames, 1004 tokens, 16 x 64, page 16, 300 frames:
+    bookkeeping of every frame bit-exact; attention on sampled frames."""
+    rows = np.unique(np.concatenate([np.arange(0, 1004, 37), [127, 128, 1003]]))
+    _stream(swa, F=300, P=1004, H=16, D=64, S=8, Wc=64, special=False, dtype=torch.bfloat16,
+            frames_to_check={0, 7, 8, 71, 72, 73, 150, 299}, check_rows=rows)
+
+
+def test_1000_frame_stream_with_specials(swa):
+    """Same cache, 1000 frames, evicted frames keep 5 special tokens each."""
+    rows = np.unique(np.concatenate([np.arange(0, 1004, 53), [0, 4, 5, 1003]]))
+    _stream(swa, F=1000, P=1004, H=16, D=64, S=8, Wc=64, special=True, dtype=torch.bfloat16,
+            frames_to_check={72, 500, 999}, check_rows=rows)
