@@ -1,0 +1,535 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the frame-causal sliding-window attention hot path.
+
+One step = one pass of every stage of the path over one batch of synthetic
+input, all inputs resident in HBM:
+  * prefill   32 frames x 1004 tokens, 16 heads x 64, window 6 frames, 8 scale
+              frames (schedule + tcgen05 attention)                  1.474 TFLOP
+  * stream    8 consecutive frames of a 300-frame-style stream at steady state:
+              append + evict on the device, split-KV attend over 8 scale + 64
+              window frames (72 x 1004 keys), combine          8 x 0.297 TFLOP
+  * band      Mistral-style token window: 32768 tokens, GQA 32/8, head_dim 128,
+              W = 4096                                               2.062 TFLOP
+  * decode    batch 64 at position 200000 against a 4096-slot rolling cache,
+              GQA 32/8, head_dim 128 (1 GiB of K/V read)         64 tokens
+``value`` is useful attention TFLOP/s over the whole step (visible query-key
+pairs x 4 x head_dim per head; masked and padded work not counted).  Per-stage
+throughput (TFLOP/s, frames/s, decode tokens/s and GB/s) is under ``parts``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torchrun; each rank runs its own shard of independent
+work (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "useful attn TFLOP/s & stream frames/s (% bf16 peak); decode tok/s (% HBM BW)"
+
+# workload ------------------------------------------------------------------
+PF = dict(F=32, P=1004, H=16, D=64, sws=6, nfpb=1, S=8)
+ST = dict(P=1004, H=16, D=64, S=8, Wc=64, page=16, frames_per_step=8)
+BD = dict(N=32768, Hq=32, Hkv=8, D=128, W=4096)
+DC = dict(B=64, W=4096, Hq=32, Hkv=8, D=128, pos=200000)
+
+CONFIG = {
+    "workload": "frame-causal SWA hot path: prefill + streaming step + token-band GQA prefill + GQA decode",
+    "prefill": "B=1, 32 frames x P=1004, C=1024 (16x64), sliding_window_size=6, num_frame_per_block=1, "
+               "num_frame_for_scale=8, bf16, LayerNorm(x)@W inputs",
+    "stream": "8 frames/step at steady state, P=1004, 16x64, 8 scale + 64 window frames, page 16, bf16",
+    "band": "32768 tokens, GQA 32/8, head_dim 128, W=4096, bf16",
+    "decode": "B=64, pos 200000 (slot 3392), 4096-slot rolling cache, GQA 32/8, head_dim 128, bf16",
+    "l2": "no flush: every stage streams inputs larger than the 126 MB L2 (197 MB, 297 MB cache, "
+          "403 MB, 1 GiB)",
+}
+
+
+def visible_frames(i, S, Wf):
+    """Frames query frame i sees: scale frames plus the frame window (causal)."""
+    lo = max(0, i - Wf + 1) if Wf > 0 else 0
+    return min(S, i + 1) + (i + 1 - max(lo, min(S, i + 1)))
+
+
+def flops_prefill():
+    Wf = PF["sws"] * PF["nfpb"]
+    pairs = sum(visible_frames(i, PF["S"], Wf) for i in range(PF["F"])) * PF["P"] ** 2
+    return pairs * PF["H"] * 4 * PF["D"]
+
+
+def flops_stream_frame():
+    keys = (ST["S"] + ST["Wc"]) * ST["P"]
+    return ST["P"] * keys * ST["H"] * 4 * ST["D"]
+
+
+def flops_band():
+    N, W = BD["N"], BD["W"]
+    pairs = sum(min(t + 1, W) for t in range(N))
+    return pairs * BD["Hq"] * 4 * BD["D"]
+
+
+def flops_decode():
+    return DC["B"] * DC["Hq"] * DC["W"] * 4 * DC["D"]
+
+
+def decode_bytes():
+    return 2 * DC["B"] * DC["W"] * DC["Hkv"] * DC["D"] * 2
+
+
+def step_flops():
+    return flops_prefill() + ST["frames_per_step"] * flops_stream_frame() + flops_band() + flops_decode()
+
+
+# peaks -----------------------------------------------------------------------
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("attn_tc.cu", "ptx.cuh", "tile_sched.h"):
+        with open(os.path.join(ROOT, "streaming_frame_causal_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# clocks ----------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"swa_clocks_{os.getpid()}_{gpu_index}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1].split()[0]))
+                    mx.append(float(parts[2].split()[0]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def gpu_smi_id(torch, dev, fallback):
+    """nvidia-smi -i accepts the GPU UUID, which survives CUDA_VISIBLE_DEVICES remapping."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(fallback)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import streaming_frame_causal_b200 as swa
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    seed = 1000 * rank
+
+    # ---- inputs (synthetic, seeded; shard = this rank's independent work)
+    pq, pk, pv = (t.to(dev) for t in synth.projected_qkv(seed=seed, F=PF["F"], P=PF["P"]))
+    pout = torch.empty_like(pq)
+    bq, bk, bv = (t.to(dev) for t in synth.band_qkv(seed=seed + 1))
+    bout = torch.empty_like(bq)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 2)
+    dq = torch.randn(DC["B"], DC["Hq"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+    dkn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+    dvn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+    dkc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+    dvc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+    dout = torch.empty_like(dq)
+    dws = torch.empty(swa.swa_decode_workspace_bytes(DC["B"], DC["Hq"], DC["Hkv"], DC["D"], DC["W"]),
+                      dtype=torch.uint8, device=dev)
+    n_pool = 16
+    frames = [tuple(torch.randn(ST["P"], ST["H"], ST["D"], generator=g, device=dev).to(torch.bfloat16)
+                    for _ in range(3)) for _ in range(n_pool)]
+    sout = torch.empty(ST["P"], ST["H"], ST["D"], dtype=torch.bfloat16, device=dev)
+    total_frames = ST["S"] + ST["Wc"] + (args.warmup + 2 * args.steps + 4) * ST["frames_per_step"]
+    cache = swa.SwaStream(num_layers=1, heads=ST["H"], head_dim=ST["D"], P=ST["P"], scale_frames=ST["S"],
+                          window_frames=ST["Wc"], page_tokens=ST["page"], max_frames=total_frames, device=dev)
+    state = {"frame": 0}
+
+    def stream_frame(fr=None):
+        i = state["frame"]
+        fq, fk, fv = frames[i % n_pool] if fr is None else fr
+        cache.swa_stream_append_evict(0, i, fk, fv)
+        cache.swa_stream_attend(0, i, fq, sout)
+        state["frame"] = i + 1
+
+    # fill the cache to steady state (8 scale + 64 window frames), untimed
+    for _ in range(ST["S"] + ST["Wc"]):
+        stream_frame()
+
+    def prefill():
+        swa.swa_prefill(pq, pk, pv, pout, S=PF["F"], P=PF["P"], sliding_window_size=PF["sws"],
+                        num_frame_per_block=PF["nfpb"], num_frame_for_scale=PF["S"])
+
+    def band():
+        swa.swa_band_prefill(bq, bk, bv, bout, window=BD["W"])
+
+    def decode():
+        swa.swa_decode(dq, dkn, dvn, dkc, dvc, DC["pos"], dout, workspace=dws)
+
+    parts = [("prefill", prefill), ("stream", lambda: [stream_frame() for _ in range(ST["frames_per_step"])]),
+             ("band", band), ("decode", decode)]
+
+    def step(evs=None):
+        for j, (_, fn) in enumerate(parts):
+            if evs is not None:
+                evs[j].record(stream)
+            fn()
+        if evs is not None:
+            evs[len(parts)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if swa.swa_device_error_check() != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    # ---- device-timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_smi_id(torch, dev, local_rank))
+    clocks.start()
+    time.sleep(0.25)
+    part_ms = {name: 0.0 for name, _ in parts}
+    launches0 = swa.swa_launch_count()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        step(ev[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = swa.swa_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    for s in range(args.steps):
+        for j, (name, _) in enumerate(parts):
+            part_ms[name] += ev[s][j].elapsed_time(ev[s][j + 1])
+    if swa.swa_device_error_check() != 0:
+        raise RuntimeError("device error flag set during the timed region")
+    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    flops = step_flops()
+    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    per = {k: v / args.steps for k, v in part_ms.items()}
+    parts_out = {
+        "prefill_tflops": flops_prefill() / (per["prefill"] * 1e-3) / 1e12,
+        "prefill_ms": per["prefill"],
+        "stream_frames_per_s": ST["frames_per_step"] / (per["stream"] * 1e-3),
+        "stream_ms_per_frame": per["stream"] / ST["frames_per_step"],
+        "stream_tflops": ST["frames_per_step"] * flops_stream_frame() / (per["stream"] * 1e-3) / 1e12,
+        "band_tflops": flops_band() / (per["band"] * 1e-3) / 1e12,
+        "band_ms": per["band"],
+        "decode_tok_per_s": DC["B"] / (per["decode"] * 1e-3),
+        "decode_us": per["decode"] * 1e3,
+        "decode_gbs": decode_bytes() / (per["decode"] * 1e-3) / 1e9,
+    }
+    parts_out["prefill_frac_of_bf16"] = parts_out["prefill_tflops"] / peaks["bf16_tflops_sustained"]
+    parts_out["band_frac_of_bf16"] = parts_out["band_tflops"] / peaks["bf16_tflops_sustained"]
+    parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
+    parts_out["decode_frac_of_hbm"] = parts_out["decode_gbs"] / peaks["hbm_gbs"]
+
+    # roofline of the dominant kernel (the single attention launch with the largest time share)
+    if per["band"] >= per["prefill"]:
+        kname, kflops, kms = "attn_tc_kernel<128> band 32768 tok GQA 32/8", flops_band(), per["band"]
+        tkey = "attn_tc_band_32768_gqa32_8_d128"
+    else:
+        kname, kflops, kms = "attn_tc_kernel<64> prefill 32x1004 16x64", flops_prefill(), per["prefill"]
+        tkey = "attn_tc_prefill_32x1004_h16_d64"
+    achieved = kflops / (kms * 1e-3) / 1e12
+    roof = {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+            "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside the step); "
+                         f"frac of burst {achieved / peaks['bf16_tflops']:.3f}",
+            "traffic": recorded_traffic(tkey)}
+
+    # ---- end to end through the public API: pinned host inputs -> device -> results back
+    e2e = run_e2e(args, swa, torch, dev, stream, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout,
+                  frames, sout, prefill, band, decode, stream_frame, world, dist)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
+        "parts": parts_out, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    return out
+
+
+def run_e2e(args, swa, torch, dev, stream, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout, frames,
+            sout, prefill, band, decode, stream_frame, world, dist):
+    """Same step, timed with every input copied from pinned host memory and
+    every output copied back inside the timed region."""
+    fps = ST["frames_per_step"]
+    h_in = [t.cpu().pin_memory() for t in (pq, pk, pv, bq, bk, bv, dq, dkn, dvn)]
+    h_frames = [tuple(t.cpu().pin_memory() for t in frames[j]) for j in range(fps)]
+    d_frames = [tuple(torch.empty_like(t) for t in frames[j]) for j in range(fps)]
+    d_in = (pq, pk, pv, bq, bk, bv, dq, dkn, dvn)
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (pout, bout, dout)]
+    h_sout = [torch.empty(sout.shape, dtype=sout.dtype, pin_memory=True) for _ in range(fps)]
+    h2d = sum(t.numel() * t.element_size() for t in h_in) + sum(
+        t.numel() * t.element_size() for fr in h_frames for t in fr)
+    d2h = sum(t.numel() * t.element_size() for t in h_out) + sum(t.numel() * t.element_size() for t in h_sout)
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        prefill()
+        h_out[0].copy_(pout, non_blocking=True)
+        for j in range(fps):
+            for h, d in zip(h_frames[j], d_frames[j]):
+                d.copy_(h, non_blocking=True)
+            stream_frame(d_frames[j])
+            h_sout[j].copy_(sout, non_blocking=True)
+        band()
+        h_out[1].copy_(bout, non_blocking=True)
+        decode()
+        h_out[2].copy_(dout, non_blocking=True)
+
+    steps = max(3, args.steps // 4)
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": world * step_flops() * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample_setup():
+    """Inputs for one bounded oracle sample of each stage (same shapes and
+    distributions as the GPU workload, generated on the host)."""
+    import numpy as np
+    import torch
+
+    import synth
+    from oracle import attention as orc
+
+    pq, pk, pv = synth.projected_qkv(seed=0, F=PF["F"], P=PF["P"])
+    pre = tuple(x[:, :, :1].float().numpy() for x in (pq, pk, pv))  # one head, all tokens
+    cache = orc.StreamCache(heads=1, head_dim=ST["D"], P=ST["P"], scale_frames=ST["S"],
+                            window_frames=ST["Wc"], page_tokens=ST["page"])
+    for i in range(ST["S"] + ST["Wc"]):
+        _, k, v = synth.stream_frame(i, P=ST["P"], H=1, D=ST["D"])
+        cache.append_evict(0, i, k.float().numpy(), v.float().numpy())
+    n_band = BD["W"] + 127
+    bq = synth.normal((1, n_band, 4, BD["D"]), 5).numpy()
+    bk = synth.normal((1, n_band, 1, BD["D"]), 6).numpy()
+    bv = synth.normal((1, n_band, 1, BD["D"]), 7).numpy()
+    dq, dkn, dvn, dkc, dvc = (x.float().numpy() for x in synth.decode_inputs(seed=1, B=1))
+    return {"orc": orc, "np": np, "synth": synth, "pre": pre, "cache": cache, "frame": ST["S"] + ST["Wc"],
+            "band": (bq, bk, bv, n_band), "dec": (dq, dkn, dvn, dkc, dvc)}
+
+
+def oracle_sample_step(ctx):
+    """One bounded oracle sample: one query frame x one head of the prefill,
+    one streaming frame (one head), 128 band rows x 4 heads, one decode
+    sequence.  Returns the useful FLOPs it computed."""
+    orc, np = ctx["orc"], ctx["np"]
+    q, k, v = ctx["pre"]
+    f = PF["F"] - 1
+    rows = np.arange(f * PF["P"], (f + 1) * PF["P"])
+    orc.prefill(q, k, v, P=PF["P"], scale_frames=PF["S"], sliding_window_size=PF["sws"],
+                num_frame_per_block=PF["nfpb"], rows=rows)
+    fl = PF["P"] * visible_frames(f, PF["S"], PF["sws"] * PF["nfpb"]) * PF["P"] * 4 * PF["D"]
+    i = ctx["frame"]
+    fq, fk, fv = ctx["synth"].stream_frame(i, P=ST["P"], H=1, D=ST["D"])
+    ctx["cache"].append_evict(0, i, fk.float().numpy(), fv.float().numpy())
+    ctx["cache"].attend(0, fq.float().numpy())
+    ctx["frame"] = i + 1
+    fl += ST["P"] * (ST["S"] + ST["Wc"]) * ST["P"] * 4 * ST["D"]
+    bq, bk, bv, n = ctx["band"]
+    rows = np.arange(n - 128, n)
+    orc.band_attention(bq, bk, bv, BD["W"], rows=rows)
+    fl += 128 * BD["W"] * 4 * BD["D"] * 4
+    dq, dkn, dvn, dkc, dvc = ctx["dec"]
+    orc.decode(dq, dkn, dvn, dkc, dvc, DC["pos"], DC["W"])
+    fl += DC["Hq"] * DC["W"] * 4 * DC["D"]
+    return fl
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s=15.0):
+    ctx = oracle_sample_setup()
+    oracle_sample_step(ctx)  # warm
+    t0 = time.perf_counter()
+    fl, n = 0, 0
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        fl += oracle_sample_step(ctx)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n} samples in {dt:.1f} s; each = 1 query frame x 1 head of the prefill, 1 stream frame "
+                      "x 1 head vs 72x1004 keys, 128 band rows x 4 heads x 4096 keys, 1 decode sequence "
+                      "x 32 heads x 4096 slots; float64 NumPy oracle"}
+
+
+def run_reference(args):
+    ctx = oracle_sample_setup()
+    for _ in range(args.warmup):
+        oracle_sample_step(ctx)
+    t0 = time.perf_counter()
+    fl = 0
+    for _ in range(args.steps):
+        fl += oracle_sample_step(ctx)
+    dt = time.perf_counter() - t0
+    value = fl / dt / 1e12
+    cores = cpu_cores()
+    sample = ("each step = 1 query frame x 1 head of the prefill, 1 stream frame x 1 head vs 72x1004 keys, "
+              "128 band rows x 4 heads x 4096 keys, 1 decode sequence x 32 heads; float64 NumPy oracle")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": CONFIG,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        if world == 1 and args.gpus > 1:
+            sys.exit("run --gpus N > 1 under torchrun (one process per GPU)")
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -216,6 +216,9 @@ swa_status swa_decode(const void* q, const void* k_new, const void* v_new,
                       int B, int Hq, int Hkv, int head_dim, void* out,
                       void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
+/* Kernel launches this library has issued in this process (all devices). */
+uint64_t swa_launch_count(void);
+
 /* ------------------------------------------------------- device errors
  * Kernels bound every wait; a wait that runs out latches a device flag and the
  * kernel returns early.  swa_device_error_check synchronizes ``stream``, reads and

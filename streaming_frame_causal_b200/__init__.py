@@ -4,8 +4,8 @@ Argument marshalling only: every function forwards tensor data pointers, sizes
 and the current CUDA stream to the C ABI of ``include/swa.h`` under the same
 name, and raises :class:`SwaError` on a non-zero status.  All arithmetic runs
 in the library's CUDA kernels; there is no fallback.  Importing this module
-fails if the library has not been built (``python -m
-streaming_frame_causal_b200.build``).
+fails if the library has not been built (``python
+streaming_frame_causal_b200/build.py``).
 
 Tensor layouts follow the pages' contracts: tokens [B, S*P, heads, head_dim]
 (the [B*S, P, C] layout with C = heads*head_dim), streaming frames
@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libswa_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "swa.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m streaming_frame_causal_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python streaming_frame_causal_b200/build.py`")
 _lib = C.CDLL(LIB_PATH)
 
 SWA_F32, SWA_BF16 = 0, 1
@@ -72,11 +72,15 @@ _sigs = {
     "swa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "swa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, C.c_longlong, _i, _i, _i, _i, _i, _vp, _vp, _sz,
                         _i, _vp]),
+    "swa_launch_count": (C.c_uint64, []),
     "swa_device_error_check": (_i, [_vp]),
     "swa_debug_wait_timeout": (_i, [_i, _vp]),
 }
 for _name, (_res, _args) in _sigs.items():
-    _f = getattr(_lib, _name)
+    try:
+        _f = getattr(_lib, _name)
+    except AttributeError as _e:
+        raise ImportError(f"{LIB_PATH} is stale (no {_name}); rebuild it") from _e
     _f.restype = _res
     _f.argtypes = _args
 
@@ -189,6 +193,11 @@ def swa_device_error_check(stream=None) -> int:
 
 def swa_debug_wait_timeout(timeout_us: int, stream=None) -> None:
     _check(_lib.swa_debug_wait_timeout(int(timeout_us), _stream(stream)), "swa_debug_wait_timeout")
+
+
+def swa_launch_count() -> int:
+    """Kernel launches the library has issued in this process."""
+    return int(_lib.swa_launch_count())
 
 
 def swa_status_str(status: int) -> str:

@@ -1,6 +1,7 @@
 """Build libswa_b200.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m streaming_frame_causal_b200.build [-v] [--force]``.  Each
+Usage: ``python streaming_frame_causal_b200/build.py [-v] [--force] [--ptxas-v]``
+(run as a file: importing the package would load the library being rebuilt).  Each
 ``csrc/*.cu`` compiles to an object under ``_build/`` (skipped when up to date),
 then the objects link into ``streaming_frame_causal_b200/libswa_b200.so``.
 """

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -17,6 +18,15 @@
 #include "tile_sched.h"
 
 using namespace swa;
+
+namespace swa {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+}  // namespace swa
+
+extern "C" uint64_t swa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ device flag
 namespace {
@@ -97,7 +107,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 swa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA; }
 
-bool tc_head_dim(int d) { return d == 64; }
+bool tc_head_dim(int d) { return d == 64 || d == 128; }
 bool simt_head_dim(int d) { return d == 32 || d == 64 || d == 128; }
 
 float scale_log2(int D) { return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D))); }

@@ -106,6 +106,7 @@ cudaError_t launch_attn_simt(const SimtParams& p, cudaStream_t stream) {
     case 128: attn_simt_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -41,14 +41,18 @@ constexpr int kSubBytes = 128 * 128;   // one 128-row x 64-column bf16 sub-tile 
 
 template <int D>
 struct Plan {
-  static_assert(D == 64, "tcgen05 path: head_dim 64 in this kernel");
+  static_assert(D == 64 || D == 128, "tcgen05 path: head_dim 64 or 128");
   static constexpr int kSubs = D / 64;                 // 64-column sub-tiles per row
   static constexpr int kTileBytes = kRows * D * 2;     // Q, K or V tile
-  static constexpr int kStages = 4;                    // K/V ring depth
-  // tensor-memory columns
+  static constexpr int kStages = (D == 64) ? 4 : 2;    // K/V ring depth
+  // Tensor-memory columns.  D = 64: S 2x128 | P 2x64 | O 2x64.  D = 128: S 2x128 |
+  // O 2x128, and P (64 columns of bf16 pairs) reuses the first half of its own
+  // S once the softmax has read S: the next QK^T that overwrites S is issued by
+  // the same thread after the PV that reads P, and tcgen05.mma operations from
+  // one thread execute in issue order.
   SWA_DEV static uint32_t col_s(int g) { return g ? 128u : 0u; }
-  SWA_DEV static uint32_t col_p(int g) { return g ? 320u : 256u; }
-  SWA_DEV static uint32_t col_o(int g) { return g ? 448u : 384u; }
+  SWA_DEV static uint32_t col_p(int g) { return D == 64 ? (g ? 320u : 256u) : col_s(g); }
+  SWA_DEV static uint32_t col_o(int g) { return D == 64 ? (g ? 448u : 384u) : (g ? 384u : 256u); }
   static constexpr uint32_t kTmemCols = 512;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
@@ -461,18 +465,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (active && ok) {
       if (__all_sync(0xffffffffu, mbar_wait(o_full, 0, p.err, ERR_WAIT_EPI))) {
         tc_fence_after();
-        uint32_t orr[D];
+        const bool store = r < w.rows[g];
+        const int row = w.row0[g] + r;
+        const float inv = 1.f / l;
+        const int64_t idx = (w.split < 0)
+                                ? (static_cast<int64_t>(w.b) * p.Nq + row) * p.Hq + w.h[g]
+                                : (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) tmem_ld32(tO + c, orr + c);
-        tmem_wait_ld();
-        if (r < w.rows[g]) {
-          const int row = w.row0[g] + r;
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c0, orr);
+          tmem_wait_ld();
+          if (!store) continue;
           if (w.split < 0) {
-            const float inv = 1.f / l;
-            __nv_bfloat16* dst =
-                reinterpret_cast<__nv_bfloat16*>(p.out) + ((static_cast<int64_t>(w.b) * p.Nq + row) * p.Hq + w.h[g]) * D;
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + idx * D + c0;
 #pragma unroll
-            for (int c = 0; c < D; c += 8) {
+            for (int c = 0; c < 32; c += 8) {
               uint4 v;
               v.x = pack_bf16x2(__uint_as_float(orr[c + 0]) * inv, __uint_as_float(orr[c + 1]) * inv);
               v.y = pack_bf16x2(__uint_as_float(orr[c + 2]) * inv, __uint_as_float(orr[c + 3]) * inv);
@@ -481,17 +489,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               *reinterpret_cast<uint4*>(dst + c) = v;
             }
           } else {
-            const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
-            float* dst = p.part_o + idx * D;
+            float* dst = p.part_o + idx * D + c0;
 #pragma unroll
-            for (int c = 0; c < D; c += 4) {
-              float4 v = make_float4(__uint_as_float(orr[c]), __uint_as_float(orr[c + 1]),
-                                     __uint_as_float(orr[c + 2]), __uint_as_float(orr[c + 3]));
-              *reinterpret_cast<float4*>(dst + c) = v;
-            }
-            p.part_ml[idx * 2 + 0] = m * sl2;
-            p.part_ml[idx * 2 + 1] = l;
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(__uint_as_float(orr[c]), __uint_as_float(orr[c + 1]),
+                              __uint_as_float(orr[c + 2]), __uint_as_float(orr[c + 3]));
           }
+        }
+        if (store && w.split >= 0) {
+          p.part_ml[idx * 2 + 0] = m * sl2;
+          p.part_ml[idx * 2 + 1] = l;
         }
       }
     } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < w.rows[g]) {
@@ -548,21 +556,33 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }  // namespace
 
 int tc_smem_bytes(int head_dim) {
-  return head_dim == 64 ? Plan<64>::kSmemBytes : -1;
+  return head_dim == 64 ? Plan<64>::kSmemBytes : head_dim == 128 ? Plan<128>::kSmemBytes : -1;
 }
 
-cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream) {
-  if (head_dim != 64) return cudaErrorInvalidValue;
-  if (n_items <= 0) return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Plan<64>::kSmemBytes);
+namespace {
+template <int D>
+cudaError_t launch_tc_d(const TcParams& p, int64_t n_items, cudaStream_t stream) {
+  static int attr_dev_mask = 0;  // devices on which the smem opt-in was set (first 31)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const int bit = 1 << (dev & 31);
+  if (!(attr_dev_mask & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               Plan<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_dev_mask |= bit;
   }
-  attn_tc_kernel<64><<<static_cast<unsigned>(n_items), kThreads, Plan<64>::kSmemBytes, stream>>>(p);
+  attn_tc_kernel<D><<<static_cast<unsigned>(n_items), kThreads, Plan<D>::kSmemBytes, stream>>>(p);
+  count_launches(1);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream) {
+  if (n_items <= 0) return cudaSuccess;
+  if (head_dim == 64) return launch_tc_d<64>(p, n_items, stream);
+  if (head_dim == 128) return launch_tc_d<128>(p, n_items, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
@@ -577,6 +597,7 @@ cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out,
     combine_kernel<128><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits);
   else
     return cudaErrorInvalidValue;
+  count_launches(1);
   return cudaGetLastError();
 }
 

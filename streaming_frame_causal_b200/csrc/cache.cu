@@ -137,11 +137,13 @@ cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
   if (blocks < 1) blocks = 1;
   if (blocks > 4096) blocks = 4096;
   append_evict_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream) {
   debug_wait_kernel<<<1, 1, 0, stream>>>(err, timeout_ns);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -280,6 +280,7 @@ cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
   if (p.D == DD && G == GG) {                                                  \
     decode_kernel<DD, GG><<<grid, kDecThreads, 0, stream>>>(p);                \
     decode_combine_kernel<DD><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);    \
+    count_launches(2);                                                         \
     return cudaGetLastError();                                                 \
   }
   SWA_DEC_CASE(128, 1) SWA_DEC_CASE(128, 2) SWA_DEC_CASE(128, 4) SWA_DEC_CASE(128, 8)
@@ -292,6 +293,7 @@ cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream) 
   const int64_t n = static_cast<int64_t>(p.B) * p.Hkv * p.D;
   const int blocks = static_cast<int>(imin(1024, static_cast<int>((n + 255) / 256)));
   decode_write_f32_kernel<<<blocks, 256, 0, stream>>>(p);
+  count_launches(1);
   return cudaGetLastError();
 }
 

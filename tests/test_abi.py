@@ -11,8 +11,8 @@ from oracle import attention as orc
 
 @pytest.fixture(scope="module")
 def swa():
-    from streaming_frame_causal_b200.build import build
-    build()
+    import __graft_entry__
+    __graft_entry__._builder().build()
     import streaming_frame_causal_b200 as m
     return m
 

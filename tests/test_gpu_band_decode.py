@@ -20,6 +20,8 @@ def swa():
     (700, 4, 2, 64, 200, torch.bfloat16),
     (520, 3, 1, 64, 130, torch.bfloat16),     # odd group size: single-head items
     (300, 4, 4, 64, 1000, torch.bfloat16),    # window wider than the sequence
+    (640, 8, 2, 128, 256, torch.bfloat16),    # head_dim 128, two query-head pairs per group
+    (333, 2, 2, 128, 64, torch.bfloat16),     # ragged last query tile, no grouping
     (200, 4, 2, 128, 50, torch.float32),
     (90, 2, 1, 32, 7, torch.float32),
 ])
@@ -69,3 +71,18 @@ def test_decode_full_workload(swa):
     check_bf16(out.float().cpu().numpy(), ref, "decode full")
     assert torch.equal(kcd[:, 3392].cpu(), kn)
     assert torch.equal(vcd[:, 3392].cpu(), vn)
+
+
+def test_band_full_workload_sampled_rows(swa):
+    """32768 tokens, GQA 32/8, D=128, window 4096: rows near the start (partial
+    windows), at the window edge and at the end, on heads of different groups."""
+    q, k, v = synth.band_qkv(seed=1)
+    out = torch.empty(q.shape, dtype=q.dtype, device="cuda")
+    swa.swa_band_prefill(q.cuda(), k.cuda(), v.cuda(), out, window=4096)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error_check() == 0
+    rows = np.array([0, 1, 127, 128, 4094, 4095, 4096, 4097, 8191, 8192, 20000, 32640, 32767])
+    heads = [0, 3, 4, 17, 31]
+    ref = orc.band_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), 4096,
+                             rows=rows, heads=heads)
+    check_bf16(out.float().cpu().numpy()[:, rows][:, :, heads], ref, "band full")

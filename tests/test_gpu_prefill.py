@@ -55,6 +55,12 @@ def test_bf16_parity_small(swa, F, P, H, sws, S, nfpb):
     check_bf16(got, _ref(q, k, v, P, S, sws, nfpb), f"bf16 F{F} P{P}")
 
 
+def test_bf16_head_dim_128(swa):
+    q, k, v = synth.tiny_qkv(seed=128, F=5, P=260, H=2, D=128, dtype=torch.bfloat16)
+    got = _run(swa, q, k, v, 5, 260, 2, 1)
+    check_bf16(got, _ref(q, k, v, 260, 1, 2), "bf16 D128")
+
+
 def test_f32_head_dims(swa):
     for D in (64, 128):
         q, k, v = synth.tiny_qkv(seed=D, F=5, P=17, H=2, D=D)
