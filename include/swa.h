@@ -216,6 +216,31 @@ swa_status swa_decode(const void* q, const void* k_new, const void* v_new,
                       int B, int Hq, int Hkv, int head_dim, void* out,
                       void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
+/* ------------------------------------------- decode without any allocation
+ * The pages have no counterpart to this entry point; it exists for callers of
+ * this library that cannot allocate device memory when they decode: a process
+ * whose device memory is fully reserved by another allocator, a host program that
+ * forbids allocation calls while it runs (cudaMalloc can synchronize the device and
+ * take unbounded time), or a plugin interface that passes inputs and outputs but
+ * offers no way to obtain memory.
+ *
+ * swa_decode_noalloc does what swa_decode does for bf16 (head_dim 64 or 128,
+ * Hq/Hkv in {1,2,4,8}) with the same arguments minus the workspace: its split-K
+ * scratch is a fixed SWA_DECODE_NOALLOC_SCRATCH_BYTES array inside the library,
+ * held on every GPU that loads the library until the process exits.  It calls no
+ * allocating routine.  Requests whose scratch would exceed the array return
+ * SWA_ERR_CAPACITY (the need is swa_decode_workspace_bytes(B, Hq, Hkv, head_dim, W));
+ * f32 or other shapes return SWA_ERR_UNSUPPORTED.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  All calls share the
+ * one array, so calls that overlap on the GPU race and must be serialized by the
+ * caller; no state from a previous call is needed or left to clear. */
+#define SWA_DECODE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+swa_status swa_decode_noalloc(const void* q, const void* k_new, const void* v_new,
+                              void* k_cache, void* v_cache, long long pos, int W,
+                              int B, int Hq, int Hkv, int head_dim, void* out,
+                              int dtype, void* stream);
+
 /* Kernel launches this library has issued in this process (all devices). */
 uint64_t swa_launch_count(void);
 

@@ -72,6 +72,7 @@ _sigs = {
     "swa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "swa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, C.c_longlong, _i, _i, _i, _i, _i, _vp, _vp, _sz,
                         _i, _vp]),
+    "swa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, C.c_longlong, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "swa_launch_count": (C.c_uint64, []),
     "swa_device_error_check": (_i, [_vp]),
     "swa_debug_wait_timeout": (_i, [_i, _vp]),
@@ -182,6 +183,17 @@ def swa_decode(q, k_new, v_new, k_cache, v_cache, pos: int, out, workspace=None,
     _check(_lib.swa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), int(pos), W,
                            B, Hq, Hkv, D, _ptr(out), _ptr(workspace), workspace.numel(),
                            _dtype_code(q), _stream(stream)), "swa_decode")
+    return out
+
+
+def swa_decode_noalloc(q, k_new, v_new, k_cache, v_cache, pos: int, out, stream=None):
+    """swa_decode for callers that cannot allocate: bf16 only, split-K scratch taken
+    from a fixed array inside the library (calls must not overlap on the GPU)."""
+    B, Hq, D = q.shape
+    W, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _check(_lib.swa_decode_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), int(pos),
+                                   W, B, Hq, Hkv, D, _ptr(out), _dtype_code(q), _stream(stream)),
+           "swa_decode_noalloc")
     return out
 
 

@@ -114,6 +114,10 @@ float scale_log2(int D) { return static_cast<float>(1.4426950408889634 / std::sq
 
 }  // namespace
 
+namespace swa {
+int* device_error_flag() { return err_ptr(); }
+}  // namespace swa
+
 // ==================================================================== status
 extern "C" const char* swa_status_str(int s) {
   switch (s) {

@@ -97,6 +97,8 @@ cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- misc
+// device address of the library's error flag on the current device (nullptr on failure)
+int* device_error_flag();
 // counts kernel launches (every launch_* helper adds what it enqueued)
 void count_launches(int n);
 cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream);
