@@ -198,28 +198,36 @@ def run_ours(args, rank, world, local_rank):
     seed = 1000 * rank
 
     # ---- inputs (synthetic, seeded; shard = this rank's independent work)
-    pq, pk, pv = (t.to(dev) for t in synth.projected_qkv(seed=seed, F=PF["F"], P=PF["P"]))
-    pout = torch.empty_like(pq)
-    bq, bk, bv = (t.to(dev) for t in synth.band_qkv(seed=seed + 1))
-    bout = torch.empty_like(bq)
+    use = (lambda s: args.stage in ("all", s))
     g = torch.Generator(device=dev)
     g.manual_seed(seed + 2)
-    dq = torch.randn(DC["B"], DC["Hq"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
-    dkn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
-    dvn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
-    dkc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
-    dvc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
-    dout = torch.empty_like(dq)
-    dws = torch.empty(swa.swa_decode_workspace_bytes(DC["B"], DC["Hq"], DC["Hkv"], DC["D"], DC["W"]),
-                      dtype=torch.uint8, device=dev)
+    pq = pk = pv = pout = bq = bk = bv = bout = dq = dkn = dvn = dkc = dvc = dout = dws = None
+    if use("prefill"):
+        pq, pk, pv = (t.to(dev) for t in synth.projected_qkv(seed=seed, F=PF["F"], P=PF["P"]))
+        pout = torch.empty_like(pq)
+    if use("band"):
+        bq, bk, bv = (t.to(dev) for t in synth.band_qkv(seed=seed + 1))
+        bout = torch.empty_like(bq)
+    if use("decode"):
+        dq = torch.randn(DC["B"], DC["Hq"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+        dkn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+        dvn = torch.randn(DC["B"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+        dkc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+        dvc = torch.randn(DC["B"], DC["W"], DC["Hkv"], DC["D"], generator=g, device=dev).to(torch.bfloat16)
+        dout = torch.empty_like(dq)
+        dws = torch.empty(swa.swa_decode_workspace_bytes(DC["B"], DC["Hq"], DC["Hkv"], DC["D"], DC["W"]),
+                          dtype=torch.uint8, device=dev)
     n_pool = 16
-    frames = [tuple(torch.randn(ST["P"], ST["H"], ST["D"], generator=g, device=dev).to(torch.bfloat16)
-                    for _ in range(3)) for _ in range(n_pool)]
-    sout = torch.empty(ST["P"], ST["H"], ST["D"], dtype=torch.bfloat16, device=dev)
-    total_frames = ST["S"] + ST["Wc"] + (args.warmup + 2 * args.steps + 4) * ST["frames_per_step"]
-    cache = swa.SwaStream(num_layers=1, heads=ST["H"], head_dim=ST["D"], P=ST["P"], scale_frames=ST["S"],
-                          window_frames=ST["Wc"], page_tokens=ST["page"], max_frames=total_frames, device=dev)
+    frames, sout, cache = [], None, None
     state = {"frame": 0}
+    if use("stream"):
+        frames = [tuple(torch.randn(ST["P"], ST["H"], ST["D"], generator=g, device=dev).to(torch.bfloat16)
+                        for _ in range(3)) for _ in range(n_pool)]
+        sout = torch.empty(ST["P"], ST["H"], ST["D"], dtype=torch.bfloat16, device=dev)
+        total_frames = ST["S"] + ST["Wc"] + (args.warmup + 2 * args.steps + 4) * ST["frames_per_step"]
+        cache = swa.SwaStream(num_layers=1, heads=ST["H"], head_dim=ST["D"], P=ST["P"], scale_frames=ST["S"],
+                              window_frames=ST["Wc"], page_tokens=ST["page"], max_frames=total_frames,
+                              device=dev)
 
     def stream_frame(fr=None):
         i = state["frame"]
@@ -228,9 +236,10 @@ def run_ours(args, rank, world, local_rank):
         cache.swa_stream_attend(0, i, fq, sout)
         state["frame"] = i + 1
 
-    # fill the cache to steady state (8 scale + 64 window frames), untimed
-    for _ in range(ST["S"] + ST["Wc"]):
-        stream_frame()
+    if use("stream"):
+        # fill the cache to steady state (8 scale + 64 window frames), untimed
+        for _ in range(ST["S"] + ST["Wc"]):
+            stream_frame()
 
     def prefill():
         swa.swa_prefill(pq, pk, pv, pout, S=PF["F"], P=PF["P"], sliding_window_size=PF["sws"],
@@ -242,8 +251,10 @@ def run_ours(args, rank, world, local_rank):
     def decode():
         swa.swa_decode(dq, dkn, dvn, dkc, dvc, DC["pos"], dout, workspace=dws)
 
-    parts = [("prefill", prefill), ("stream", lambda: [stream_frame() for _ in range(ST["frames_per_step"])]),
-             ("band", band), ("decode", decode)]
+    all_parts = [("prefill", prefill),
+                 ("stream", lambda: [stream_frame() for _ in range(ST["frames_per_step"])]),
+                 ("band", band), ("decode", decode)]
+    parts = [(n, fn) for n, fn in all_parts if use(n)]
 
     def step(evs=None):
         for j, (_, fn) in enumerate(parts):
@@ -291,85 +302,111 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     elapsed_ms = float(t.item())
     ms_per_step = elapsed_ms / args.steps
-    flops = step_flops()
+    stage_flops = {"prefill": flops_prefill(), "stream": ST["frames_per_step"] * flops_stream_frame(),
+                   "band": flops_band(), "decode": flops_decode()}
+    flops = sum(stage_flops[n] for n, _ in parts)
     value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
 
     peaks = measured_peaks()
     per = {k: v / args.steps for k, v in part_ms.items()}
-    parts_out = {
-        "prefill_tflops": flops_prefill() / (per["prefill"] * 1e-3) / 1e12,
-        "prefill_ms": per["prefill"],
-        "stream_frames_per_s": ST["frames_per_step"] / (per["stream"] * 1e-3),
-        "stream_ms_per_frame": per["stream"] / ST["frames_per_step"],
-        "stream_tflops": ST["frames_per_step"] * flops_stream_frame() / (per["stream"] * 1e-3) / 1e12,
-        "band_tflops": flops_band() / (per["band"] * 1e-3) / 1e12,
-        "band_ms": per["band"],
-        "decode_tok_per_s": DC["B"] / (per["decode"] * 1e-3),
-        "decode_us": per["decode"] * 1e3,
-        "decode_gbs": decode_bytes() / (per["decode"] * 1e-3) / 1e9,
-    }
-    parts_out["prefill_frac_of_bf16"] = parts_out["prefill_tflops"] / peaks["bf16_tflops_sustained"]
-    parts_out["band_frac_of_bf16"] = parts_out["band_tflops"] / peaks["bf16_tflops_sustained"]
-    parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
-    parts_out["decode_frac_of_hbm"] = parts_out["decode_gbs"] / peaks["hbm_gbs"]
+    parts_out = {}
+    if "prefill" in per:
+        parts_out["prefill_tflops"] = flops_prefill() / (per["prefill"] * 1e-3) / 1e12
+        parts_out["prefill_ms"] = per["prefill"]
+        parts_out["prefill_frac_of_bf16"] = parts_out["prefill_tflops"] / peaks["bf16_tflops_sustained"]
+    if "stream" in per:
+        parts_out["stream_frames_per_s"] = ST["frames_per_step"] / (per["stream"] * 1e-3)
+        parts_out["stream_ms_per_frame"] = per["stream"] / ST["frames_per_step"]
+        parts_out["stream_tflops"] = stage_flops["stream"] / (per["stream"] * 1e-3) / 1e12
+        parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
+    if "band" in per:
+        parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
+        parts_out["band_ms"] = per["band"]
+        parts_out["band_frac_of_bf16"] = parts_out["band_tflops"] / peaks["bf16_tflops_sustained"]
+    if "decode" in per:
+        parts_out["decode_tok_per_s"] = DC["B"] / (per["decode"] * 1e-3)
+        parts_out["decode_us"] = per["decode"] * 1e3
+        parts_out["decode_gbs"] = decode_bytes() / (per["decode"] * 1e-3) / 1e9
+        parts_out["decode_frac_of_hbm"] = parts_out["decode_gbs"] / peaks["hbm_gbs"]
 
     # roofline of the dominant kernel (the single attention launch with the largest time share)
-    if per["band"] >= per["prefill"]:
-        kname, kflops, kms = "attn_tc_kernel<128> band 32768 tok GQA 32/8", flops_band(), per["band"]
-        tkey = "attn_tc_band_32768_gqa32_8_d128"
+    cands = []
+    if "band" in per:
+        cands.append((per["band"], "attn_tc_kernel<128> band 32768 tok GQA 32/8", flops_band(),
+                      "attn_tc_band_32768_gqa32_8_d128", "tensor"))
+    if "prefill" in per:
+        cands.append((per["prefill"], "attn_tc_kernel<64> prefill 32x1004 16x64", flops_prefill(),
+                      "attn_tc_prefill_32x1004_h16_d64", "tensor"))
+    if "stream" in per:
+        cands.append((per["stream"], "attn_tc_kernel<64> stream attend + append + combine, 8 frames",
+                      stage_flops["stream"], "attn_tc_stream_72x1004_h16_d64", "tensor"))
+    if "decode" in per:
+        cands.append((per["decode"], "decode_kernel<128,4> B64 W4096", decode_bytes(),
+                      "decode_b64_w4096_gqa32_8_d128", "hbm"))
+    kms, kname, kwork, tkey, bound = max(cands)
+    if bound == "tensor":
+        achieved = kwork / (kms * 1e-3) / 1e12
+        roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside the step); "
+                             f"frac of burst {achieved / peaks['bf16_tflops']:.3f}",
+                "traffic": recorded_traffic(tkey)}
     else:
-        kname, kflops, kms = "attn_tc_kernel<64> prefill 32x1004 16x64", flops_prefill(), per["prefill"]
-        tkey = "attn_tc_prefill_32x1004_h16_d64"
-    achieved = kflops / (kms * 1e-3) / 1e12
-    roof = {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
-            "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside the step); "
-                         f"frac of burst {achieved / peaks['bf16_tflops']:.3f}",
-            "traffic": recorded_traffic(tkey)}
+        achieved = kwork / (kms * 1e-3) / 1e9
+        roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_note": f"{peaks['source']} HBM copy bandwidth",
+                "traffic": recorded_traffic(tkey)}
 
     # ---- end to end through the public API: pinned host inputs -> device -> results back
-    e2e = run_e2e(args, swa, torch, dev, stream, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout,
-                  frames, sout, prefill, band, decode, stream_frame, world, dist)
+    e2e = run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn,
+                  dout, frames, sout, prefill, band, decode, stream_frame, world, dist, flops)
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": CONFIG if args.stage == "all" else dict(CONFIG, stage_only=args.stage),
         "parts": parts_out, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clk,
     }
     return out
 
 
-def run_e2e(args, swa, torch, dev, stream, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout, frames,
-            sout, prefill, band, decode, stream_frame, world, dist):
+def run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout,
+            frames, sout, prefill, band, decode, stream_frame, world, dist, flops):
     """Same step, timed with every input copied from pinned host memory and
     every output copied back inside the timed region."""
     fps = ST["frames_per_step"]
-    h_in = [t.cpu().pin_memory() for t in (pq, pk, pv, bq, bk, bv, dq, dkn, dvn)]
-    h_frames = [tuple(t.cpu().pin_memory() for t in frames[j]) for j in range(fps)]
-    d_frames = [tuple(torch.empty_like(t) for t in frames[j]) for j in range(fps)]
-    d_in = (pq, pk, pv, bq, bk, bv, dq, dkn, dvn)
-    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (pout, bout, dout)]
-    h_sout = [torch.empty(sout.shape, dtype=sout.dtype, pin_memory=True) for _ in range(fps)]
+    names = {n for n, _ in parts}
+    d_in = [t for t in (pq, pk, pv, bq, bk, bv, dq, dkn, dvn) if t is not None]
+    h_in = [t.cpu().pin_memory() for t in d_in]
+    use_stream = "stream" in names
+    h_frames = [tuple(t.cpu().pin_memory() for t in frames[j]) for j in range(fps)] if use_stream else []
+    d_frames = [tuple(torch.empty_like(t) for t in frames[j]) for j in range(fps)] if use_stream else []
+    d_out = [t for t in (pout, bout, dout) if t is not None]
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
+    h_sout = [torch.empty(sout.shape, dtype=sout.dtype, pin_memory=True) for _ in range(fps)] if use_stream else []
     h2d = sum(t.numel() * t.element_size() for t in h_in) + sum(
         t.numel() * t.element_size() for fr in h_frames for t in fr)
     d2h = sum(t.numel() * t.element_size() for t in h_out) + sum(t.numel() * t.element_size() for t in h_sout)
+    outs = dict(zip([n for n, t in (("prefill", pout), ("band", bout), ("decode", dout)) if t is not None],
+                    zip(d_out, h_out)))
 
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        prefill()
-        h_out[0].copy_(pout, non_blocking=True)
-        for j in range(fps):
-            for h, d in zip(h_frames[j], d_frames[j]):
-                d.copy_(h, non_blocking=True)
-            stream_frame(d_frames[j])
-            h_sout[j].copy_(sout, non_blocking=True)
-        band()
-        h_out[1].copy_(bout, non_blocking=True)
-        decode()
-        h_out[2].copy_(dout, non_blocking=True)
+        for name, fn in parts:
+            if name == "stream":
+                for j in range(fps):
+                    for h, d in zip(h_frames[j], d_frames[j]):
+                        d.copy_(h, non_blocking=True)
+                    stream_frame(d_frames[j])
+                    h_sout[j].copy_(sout, non_blocking=True)
+            else:
+                fn()
+                d, h = outs[name]
+                h.copy_(d, non_blocking=True)
 
     steps = max(3, args.steps // 4)
     e2e_step()
@@ -388,7 +425,7 @@ def run_e2e(args, swa, torch, dev, stream, pq, pk, pv, pout, bq, bk, bv, bout, d
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
-    return {"value": world * step_flops() * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": world * flops * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": ms / steps}
 
@@ -497,6 +534,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=("all", "prefill", "stream", "band", "decode"), default="all",
+                    help="time one stage only (for profiling); the reported value then covers that stage")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -523,7 +562,7 @@ def main():
     try:
         out = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and args.stage == "all":
                 out["cpu_baseline"] = cpu_baseline()
             print(json.dumps(out), flush=True)
     finally:
