@@ -241,6 +241,11 @@ swa_status swa_decode_noalloc(const void* q, const void* k_new, const void* v_ne
                               int B, int Hq, int Hkv, int head_dim, void* out,
                               int dtype, void* stream);
 
+/* Diagnostic: y[i] = 2^x[i] as the attention kernels' FMA-pipe polynomial computes it
+ * (Cody-Waite reduction + fitted cubic, relative error <= 8e-5 for x >= -125), for
+ * n float32 device values.  Lets tests compare it with the hardware exp2. */
+swa_status swa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
+
 /* Kernel launches this library has issued in this process (all devices). */
 uint64_t swa_launch_count(void);
 

@@ -76,6 +76,7 @@ _sigs = {
     "swa_launch_count": (C.c_uint64, []),
     "swa_device_error_check": (_i, [_vp]),
     "swa_debug_wait_timeout": (_i, [_i, _vp]),
+    "swa_debug_exp2_poly": (_i, [_vp, _vp, _i, _vp]),
 }
 for _name, (_res, _args) in _sigs.items():
     try:
@@ -210,6 +211,12 @@ def swa_debug_wait_timeout(timeout_us: int, stream=None) -> None:
 def swa_launch_count() -> int:
     """Kernel launches the library has issued in this process."""
     return int(_lib.swa_launch_count())
+
+
+def swa_debug_exp2_poly(x, y, stream=None):
+    """y = 2^x through the kernels' FMA-pipe polynomial (float32 device tensors)."""
+    _check(_lib.swa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "swa_debug_exp2_poly")
+    return y
 
 
 def swa_status_str(status: int) -> str:

@@ -703,3 +703,10 @@ extern "C" swa_status swa_debug_wait_timeout(int timeout_us, void* stream) {
   if (!err) return SWA_ERR_CUDA;
   return cuda_status(launch_debug_wait(err, static_cast<long long>(timeout_us) * 1000, static_cast<cudaStream_t>(stream)));
 }
+
+extern "C" swa_status swa_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return SWA_ERR_ARG;
+  if (n == 0) return SWA_OK;
+  if (!x || !y) return SWA_ERR_ARG;
+  return cuda_status(launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
+}

@@ -8,11 +8,15 @@
 // frames are visible; "KV Cache Eviction Strategy": only retained frames are in
 // the cache; sliding-window explainer: token band t-W+1..t).
 //
-// CTA organisation (320 threads, one CTA per SM):
+// CTA organisation (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q tiles once, then K/V key tiles into a ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 2-5   softmax for query tile A (one thread per query row)
-//   warps 6-9   softmax for query tile B
+//   warps 2-3   idle
+//   warps 4-7   softmax for query tile A (one thread per query row)
+//   warps 8-11  softmax for query tile B
+// After set-up, warpgroup 0 gives registers back (setmaxnreg.dec to 64) and the
+// softmax warpgroups take them (setmaxnreg.inc to 216), so a thread can hold a
+// whole 128-column row of S in registers.
 // The two query tiles ping-pong: while softmax A turns S_A into P_A, the tensor
 // core runs P_B V and Q_B K^T, and the other way round.  S (f32, 128 columns),
 // P (bf16 pairs, 64 columns) and O (f32, D columns) of each tile live in tensor
@@ -28,6 +32,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "tile_sched.h"
 
@@ -35,7 +40,12 @@ namespace swa {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;     // 3 warpgroups
+constexpr int kRegsLaunch = 168;  // registers per thread at launch (384 x 168 = 64512 of 65536)
+constexpr int kRegsCtl = 64;      // warpgroup 0 (TMA producer, MMA issuer) after setmaxnreg.dec
+constexpr int kRegsSoftmax = 216; // warpgroups 1-2 (softmax) after setmaxnreg.inc
+static_assert(4 * kRegsCtl + 8 * kRegsSoftmax <= 12 * kRegsLaunch,
+              "register split must fit the pool the CTA was launched with");
 constexpr int kRows = kTileRows;       // 128
 constexpr int kSubBytes = 128 * 128;   // one 128-row x 64-column bf16 sub-tile (16 KB)
 
@@ -66,17 +76,17 @@ struct Plan {
 
 struct Work {
   int b, kvh;
-  int h[2];
-  int row0[2];   // first query row of each tile (row index in the Q tensor, per batch)
-  int rows[2];   // valid query rows (0 = tile absent)
-  int t_begin, t_end;
-  int split;     // >= 0: write split-KV partials; -1: write the final output
+  int h0, h1;          // query heads of tiles A and B
+  int qrow0, qrow1;    // first query row of tiles A and B (row index in the Q tensor, per batch)
+  int rows0, rows1;    // valid query rows (0 = tile absent)
+  int t_begin, t_end;  // key-tile range of this item
+  int split;           // >= 0: write split-KV partials; -1: write the final output
   int nseg;
-  int lrow[2], llen[2];
-  const int* grow;
+  int srow0, slen0, srow1, slen1;  // inline key runs (frame and band modes)
+  const int* grow;                 // key runs in device metadata (stream mode)
   const int* glen;
-  SWA_DEV int seg_row(int s) const { return grow ? __ldg(grow + s) : lrow[s]; }
-  SWA_DEV int seg_len(int s) const { return glen ? __ldg(glen + s) : llen[s]; }
+  SWA_DEV int seg_row(int s) const { return grow ? __ldg(grow + s) : (s == 0 ? srow0 : srow1); }
+  SWA_DEV int seg_len(int s) const { return glen ? __ldg(glen + s) : (s == 0 ? slen0 : slen1); }
 };
 
 struct Cursor {
@@ -124,22 +134,25 @@ SWA_DEV Work decode_work(const TcParams& p) {
   w.glen = nullptr;
   w.split = -1;
   w.nseg = 0;
+  w.srow0 = w.slen0 = w.srow1 = w.slen1 = 0;
   const int64_t bid = blockIdx.x;
   if (p.mode == TC_FRAME) {
     const PrefillItem it = prefill_item(bid, p.B, p.Hq, p.F, p.n_pairs);
     w.b = it.b;
     w.kvh = it.h / (p.Hq / p.Hkv);
-    w.h[0] = w.h[1] = it.h;
+    w.h0 = w.h1 = it.h;
     const int t0 = 2 * it.pair;
-    w.rows[0] = qtile_rows(p.P, t0);
-    w.rows[1] = qtile_rows(p.P, t0 + 1);
-    w.row0[0] = it.f * p.P + t0 * kRows;
-    w.row0[1] = w.row0[0] + kRows;
+    w.rows0 = qtile_rows(p.P, t0);
+    w.rows1 = qtile_rows(p.P, t0 + 1);
+    w.qrow0 = it.f * p.P + t0 * kRows;
+    w.qrow1 = w.qrow0 + kRows;
     int lo[2], hi[2];
     w.nseg = frame_intervals(it.f, p.Wf, p.S, lo, hi);
-    for (int s = 0; s < w.nseg; ++s) {
-      w.lrow[s] = lo[s] * p.P;
-      w.llen[s] = (hi[s] - lo[s]) * p.P;
+    w.srow0 = lo[0] * p.P;
+    w.slen0 = (hi[0] - lo[0]) * p.P;
+    if (w.nseg > 1) {
+      w.srow1 = lo[1] * p.P;
+      w.slen1 = (hi[1] - lo[1]) * p.P;
     }
     w.t_begin = 0;
     w.t_end = total_tiles(w);
@@ -149,28 +162,28 @@ SWA_DEV Work decode_work(const TcParams& p) {
     w.kvh = it.kvh;
     const int t0 = it.t * kRows;
     const int rows = imin(kRows, p.Nq - t0);
-    w.h[0] = it.h0;
-    w.h[1] = it.h1 < 0 ? it.h0 : it.h1;
-    w.row0[0] = w.row0[1] = t0;
-    w.rows[0] = rows;
-    w.rows[1] = it.h1 < 0 ? 0 : rows;
+    w.h0 = it.h0;
+    w.h1 = it.h1 < 0 ? it.h0 : it.h1;
+    w.qrow0 = w.qrow1 = t0;
+    w.rows0 = rows;
+    w.rows1 = it.h1 < 0 ? 0 : rows;
     int lo, hi;
     band_keys(t0, rows, p.W, &lo, &hi);
     w.nseg = 1;
-    w.lrow[0] = lo;
-    w.llen[0] = hi - lo;
+    w.srow0 = lo;
+    w.slen0 = hi - lo;
     w.t_begin = 0;
     w.t_end = total_tiles(w);
   } else {  // TC_STREAM
     const StreamItem it = stream_item(bid, p.Hq, p.n_pairs);
     w.b = 0;
     w.kvh = it.h / (p.Hq / p.Hkv);
-    w.h[0] = w.h[1] = it.h;
+    w.h0 = w.h1 = it.h;
     const int t0 = 2 * it.pair;
-    w.rows[0] = qtile_rows(p.P, t0);
-    w.rows[1] = qtile_rows(p.P, t0 + 1);
-    w.row0[0] = t0 * kRows;
-    w.row0[1] = w.row0[0] + kRows;
+    w.rows0 = qtile_rows(p.P, t0);
+    w.rows1 = qtile_rows(p.P, t0 + 1);
+    w.qrow0 = t0 * kRows;
+    w.qrow1 = w.qrow0 + kRows;
     w.grow = p.seg_row;
     w.glen = p.seg_len;
     const int n = __ldg(p.meta_hdr + 5);
@@ -182,21 +195,14 @@ SWA_DEV Work decode_work(const TcParams& p) {
   return w;
 }
 
-// Masked columns of a 64-column chunk of S become -inf: the unused tail of the
-// last tile of a key run (``cut``), or outside the band t-W+1..t.
-SWA_DEV void mask_cols(uint32_t* x, int c0, bool cut, bool band_edge, int kvalid, int krow, int qrow, int W) {
-  if (cut) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-      if (c0 + c >= kvalid) x[c] = __float_as_uint(-INFINITY);
-  } else if (band_edge) {
-    const int lo = qrow - W + 1;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const int key = krow + c0 + c;
-      if (c0 + c >= kvalid || key < lo || key > qrow) x[c] = __float_as_uint(-INFINITY);
-    }
-  }
+#ifndef SWA_POLY_PAIRS
+#define SWA_POLY_PAIRS 3  // of every 8 column pairs, how many take 2^x on the FMA pipe
+#endif
+
+SWA_DEV float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 template <int D>
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const Work w = decode_work(p);
   const int T = w.t_end - w.t_begin;
-  const bool has_b = w.rows[1] > 0;
+  const bool has_b = w.rows1 > 0;
 
   // barriers
   const uint32_t bar0 = base + PL::kOffBar;
@@ -248,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + PL::kOffTmem);
-
+  if (warp < 4) {
+  reg_dealloc<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && T > 0) {
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mbar_arrive_expect_tx(q_full(g), PL::kTileBytes);
         for (int sub = 0; sub < PL::kSubs; ++sub)
           tma_load_4d(base + PL::kOffQ + g * PL::kTileBytes + sub * kSubBytes, &p.tm_q, q_full(g),
-                      sub * 64, w.h[g], w.row0[g], w.b);
+                      sub * 64, g ? w.h1 : w.h0, g ? w.qrow1 : w.qrow0, w.b);
       }
       Cursor cur;
       bool ok = cursor_seek(w, w.t_begin, cur);
@@ -361,9 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mma_commit(drain);
       mbar_wait(drain, 0, p.err, ERR_WAIT_MMA);
     }
+  }
   } else {
+    reg_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int g = (warp - 2) >> 2;  // 0: tile A, 1: tile B
+    const int g = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -372,9 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t tO = tmem + lane_off + PL::col_o(g);
     const float sl2 = p.scale_log2;
     const bool band = (p.mode == TC_BAND);
-    const int qrow = w.row0[g] + r;  // query token (band mode: absolute position)
-    float m = -INFINITY;             // running max of raw scores
-    float l = 0.f;                   // running row sum (relative to m)
+    const int my_h = g ? w.h1 : w.h0;
+    const int my_row0 = g ? w.qrow1 : w.qrow0;
+    const int my_rows = g ? w.rows1 : w.rows0;
+    const int qrow = my_row0 + r;  // query token (band mode: absolute position)
+    float m = -INFINITY;           // running reference max of raw scores
+    float l = 0.f;                 // running row sum relative to m
     bool ok = (g == 0 || has_b) && T > 0;
     const bool active = ok;
     Cursor cur;
@@ -392,26 +404,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         break;
       }
       tc_fence_after();
-      // ---- pass 1: row max over the tile (masked columns excluded)
-      const bool band_edge =
-          band && !((krow >= w.row0[g] + w.rows[g] - 1 - p.W + 1) && (krow + kvalid - 1 <= w.row0[g]) &&
-                    kvalid == kRows);
-      const bool cut = !band && kvalid < kRows;
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      uint32_t s[128];
+      tmem_ld32(tS + 0, s);
+      tmem_ld32(tS + 32, s + 32);
+      tmem_ld32(tS + 64, s + 64);
+      tmem_ld32(tS + 96, s + 96);
+      tmem_wait_ld();
+      // ---- masks: unused tail of the last tile of a key run, band edges
+      if (band) {
+        const bool inside = (krow >= my_row0 + my_rows - 1 - p.W + 1) && (krow + kvalid - 1 <= my_row0) &&
+                            kvalid == kRows;
+        if (!inside) {
+          const int lo = qrow - p.W + 1;
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 64) {
-        uint32_t x[64];
-        tmem_ld32(tS + c0, x);
-        tmem_ld32(tS + c0 + 32, x + 32);
-        tmem_wait_ld();
-        mask_cols(x, c0, cut, band_edge, kvalid, krow, qrow, p.W);
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(x[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(x[c + 1]));
+          for (int c = 0; c < 128; ++c) {
+            const int key = krow + c;
+            if (c >= kvalid || key < lo || key > qrow) s[c] = __float_as_uint(-INFINITY);
+          }
         }
+      } else if (kvalid < kRows) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= kvalid) s[c] = __float_as_uint(-INFINITY);
       }
-      const float tmax = fmaxf(mx0, mx1);
+      // ---- row max: eight independent 3-input max chains
+      float a[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = max3f(__uint_as_float(s[k]), __uint_as_float(s[8 + k]), __uint_as_float(s[16 + k]));
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          a[k] = max3f(a[k], __uint_as_float(s[c + k]), __uint_as_float(s[c + 8 + k]));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], __uint_as_float(s[120 + k]));
+      const float tmax = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
       const float m_new = fmaxf(m, tmax);
       const bool grow = (m != -INFINITY) && ((m_new - m) * sl2 > 8.0f);
       float alpha = 1.f;
@@ -436,27 +464,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tmem_wait_st();
       }
       l *= alpha;
-      // ---- pass 2: P = 2^(s*scale - m*scale) as bf16 pairs into TMEM
+      // ---- P = 2^(s*scale - m*scale): MUFU for most column pairs, the
+      // polynomial on the FMA pipe for SWA_POLY_PAIRS of every 8; packed bf16
+      // pairs overwrite the front of s (pair pi reads s[2pi], s[2pi+1] >= pi)
       const float nb = (m == -INFINITY) ? 0.f : -m * sl2;
-      float sum0 = 0.f, sum1 = 0.f;
+      const float2 c2 = make_float2(sl2, sl2);
+      const float2 nb2 = make_float2(nb, nb);
+      float2 acc[4];
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 64) {
-        uint32_t x[64];
-        tmem_ld32(tS + c0, x);
-        tmem_ld32(tS + c0 + 32, x + 32);
-        tmem_wait_ld();
-        mask_cols(x, c0, cut, band_edge, kvalid, krow, qrow, p.W);
+      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(x[c]), sl2, nb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(x[c + 1]), sl2, nb));
-          sum0 += p0;
-          sum1 += p1;
-          x[c >> 1] = pack_bf16x2(p0, p1);  // index c/2 <= c: already consumed
+      for (int pi = 0; pi < 64; ++pi) {
+        const float2 x =
+            __ffma2_rn(make_float2(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])), c2, nb2);
+        float2 pr;
+        if ((pi & 7) < SWA_POLY_PAIRS) {
+          pr = exp2_poly2(x);
+        } else {
+          pr.x = ex2_approx(x.x);
+          pr.y = ex2_approx(x.y);
         }
-        tmem_st32(tP + (c0 >> 1), x);
+        acc[pi & 3] = __fadd2_rn(acc[pi & 3], pr);
+        s[pi] = pack_bf16x2(pr.x, pr.y);
       }
-      l += sum0 + sum1;
+      l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+      tmem_st32(tP + 0, s);
+      tmem_st32(tP + 32, s + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full(g));
@@ -465,12 +498,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (active && ok) {
       if (__all_sync(0xffffffffu, mbar_wait(o_full, 0, p.err, ERR_WAIT_EPI))) {
         tc_fence_after();
-        const bool store = r < w.rows[g];
-        const int row = w.row0[g] + r;
+        const bool store = r < my_rows;
+        const int row = my_row0 + r;
         const float inv = 1.f / l;
         const int64_t idx = (w.split < 0)
-                                ? (static_cast<int64_t>(w.b) * p.Nq + row) * p.Hq + w.h[g]
-                                : (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
+                                ? (static_cast<int64_t>(w.b) * p.Nq + row) * p.Hq + my_h
+                                : (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t orr[32];
@@ -502,10 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           p.part_ml[idx * 2 + 1] = l;
         }
       }
-    } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < w.rows[g]) {
+    } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < my_rows) {
       // empty split: contributes nothing to the combine
-      const int row = w.row0[g] + r;
-      const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + w.h[g];
+      const int row = my_row0 + r;
+      const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
       p.part_ml[idx * 2 + 0] = -INFINITY;
       p.part_ml[idx * 2 + 1] = 0.f;
     }
@@ -567,8 +600,14 @@ cudaError_t launch_tc_d(const TcParams& p, int64_t n_items, cudaStream_t stream)
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const int bit = 1 << (dev & 31);
   if (!(attr_dev_mask & bit)) {
-    const cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               Plan<D>::kSmemBytes);
+    // the setmaxnreg split moves registers inside the pool the CTA is launched
+    // with; refuse to launch a build whose pool would be too small (the
+    // increasing warpgroups would otherwise wait forever)
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * 12 < 4 * kRegsCtl + 8 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_dev_mask |= bit;
   }

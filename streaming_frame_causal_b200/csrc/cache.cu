@@ -21,6 +21,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "tile_sched.h"
 
@@ -129,7 +130,26 @@ __global__ void debug_wait_kernel(int* err, long long timeout_ns) {
   }
 }
 
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  if (pairs == 0) return cudaSuccess;
+  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
+  count_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
   const int64_t work = 2LL * p.P * (p.row_bytes >> 4);

@@ -101,6 +101,7 @@ cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);
 int* device_error_flag();
 // counts kernel launches (every launch_* helper adds what it enqueued)
 void count_launches(int n);
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream);
 
 }  // namespace swa

@@ -95,6 +95,17 @@ SWA_DEV void tma_load_4d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, 
       : "memory");
 }
 
+// ------------------------------------------------------------------ registers
+// Move registers between warpgroups (every thread of the warpgroup executes it).
+template <int N>
+SWA_DEV void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+SWA_DEV void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ tcgen05
 SWA_DEV void tmem_alloc(uint32_t smem_dst, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst),
