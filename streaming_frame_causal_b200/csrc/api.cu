@@ -105,6 +105,23 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B) 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+bool swa::encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), 1, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
 swa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA; }
 
 bool tc_head_dim(int d) { return d == 64 || d == 128; }
@@ -357,7 +374,6 @@ extern "C" swa_status swa_decode(const void* q, const void* k_new, const void* v
   if (!workspace || workspace_bytes < need) return SWA_ERR_CAPACITY;
   if (!aligned16(workspace)) return SWA_ERR_ARG;
   p.chunks = decode_chunks(B, Hkv, W);
-  p.chunk_len = cdiv(p.n_valid, p.chunks);
   const size_t n_part = static_cast<size_t>(B) * Hkv * p.chunks * G;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = p.part_o + n_part * head_dim;

@@ -21,6 +21,8 @@
 #include <cmath>
 #include <cstdint>
 
+#include <cuda.h>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_sched.h"
@@ -28,127 +30,190 @@
 namespace swa {
 namespace {
 
-constexpr int kDecThreads = 128;   // 4 warps x 4 row-groups = 16 rows per step
-constexpr int kRowsPerStep = 16;
+constexpr int kDecThreads = 128;  // 4 warps; each warp covers 4 rows per pass (8 lanes per row)
+constexpr int kDecRows = 32;      // cache rows per pipeline stage
+constexpr int kDecStages = 4;     // stages in flight per CTA
 
 SWA_DEV float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 SWA_DEV float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
-SWA_DEV uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+SWA_DEV void unpack8(const uint4 u, float2* f) {
+  f[0] = make_float2(bf_lo(u.x), bf_hi(u.x));
+  f[1] = make_float2(bf_lo(u.y), bf_hi(u.y));
+  f[2] = make_float2(bf_lo(u.z), bf_hi(u.z));
+  f[3] = make_float2(bf_lo(u.w), bf_hi(u.w));
 }
 
+SWA_DEV void tma_load_3d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+      : "memory");
+}
+
+template <int D>
+struct DecPlan {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kTileBytes = kDecRows * kRowBytes;  // K (or V) rows of one stage
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kDecStages * kTileBytes;
+  static constexpr int kOffBar = 2 * kDecStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 128;
+};
+
+// Lane (grp, sub) of a warp handles row grp of each 4-row pass and owns head_dim
+// elements [64v + 8 sub, 64v + 8 sub + 8) for v < D/64: its 16-byte reads of a
+// row then hit 8 distinct bank quads, so a warp's read of 4 rows takes the
+// minimum 4 shared-memory wavefronts.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeParams p) {
-  constexpr int EL = D / 8;   // head_dim elements per lane
-  constexpr int NV = EL / 8;  // 16-byte vectors per lane per row
+__global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
+  using PL = DecPlan<D>;
+  constexpr int NV = D / 64;  // 16-byte chunks per lane per row
+  extern __shared__ __align__(128) uint8_t dsm[];
   const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane >> 3, sub = lane & 7;
   const int t_begin = c * p.chunk_len;
   const int t_end = imin(t_begin + p.chunk_len, p.n_valid);
+  const int n_st = t_end > t_begin ? cdiv(t_end - t_begin, kDecRows) : 0;
+  const uint32_t sbase = smem_u32(dsm);
+  const uint32_t bar_full = sbase + PL::kOffBar;
+  const uint32_t bar_empty = bar_full + 8 * kDecStages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int i) {
+    const int s = i % kDecStages;
+    const int row = b * p.W + t_begin + i * kDecRows;
+    mbar_arrive_expect_tx(bar_full + 8 * s, 2 * PL::kTileBytes);
+    tma_load_3d(sbase + PL::kOffK + s * PL::kTileBytes, &p.tm_k, bar_full + 8 * s, 0, kvh, row);
+    tma_load_3d(sbase + PL::kOffV + s * PL::kTileBytes, &p.tm_v, bar_full + 8 * s, 0, kvh, row);
+  };
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    for (int i = 0; i < imin(kDecStages, n_st); ++i) issue(i);
+  }
 
   const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q);
-  float2 q[G][EL / 2];
+  float2 q[G][4 * NV];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16* qp = qb + (static_cast<int64_t>(b) * p.Hq + kvh * G + g) * D + sub * EL;
+    const __nv_bfloat16* qp = qb + (static_cast<int64_t>(b) * p.Hq + kvh * G + g) * D + sub * 8;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-      const uint4 u = *reinterpret_cast<const uint4*>(qp + v * 8);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      unpack8(*reinterpret_cast<const uint4*>(qp + v * 64), &q[g][4 * v]);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        q[g][v * 4 + e] = make_float2(bf_lo(w[e]) * p.scale_log2, bf_hi(w[e]) * p.scale_log2);
+        q[g][4 * v + e] = make_float2(q[g][4 * v + e].x * p.scale_log2, q[g][4 * v + e].y * p.scale_log2);
     }
   }
-  float2 o[G][EL / 2];
+  float2 o[G][4 * NV];
   float m[G], l[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m[g] = -INFINITY;
     l[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < EL / 2; ++e) o[g][e] = make_float2(0.f, 0.f);
+    for (int e = 0; e < 4 * NV; ++e) o[g][e] = make_float2(0.f, 0.f);
   }
-
   const int64_t row_elems = static_cast<int64_t>(p.Hkv) * D;
-  const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.k_cache) +
-                            static_cast<int64_t>(b) * p.W * row_elems + kvh * D + sub * EL;
-  const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.v_cache) +
-                            static_cast<int64_t>(b) * p.W * row_elems + kvh * D + sub * EL;
-  const int64_t new_off = (static_cast<int64_t>(b) * p.Hkv + kvh) * D + sub * EL;
+  const int64_t new_off = (static_cast<int64_t>(b) * p.Hkv + kvh) * D + sub * 8;
+  bool ok = true;
 
-  // rows t_begin + 16k + tl; the loop bound is warp-uniform so the group
-  // reductions below always see all 32 lanes
-  for (int tb = t_begin + warp * 4; tb < t_end; tb += kRowsPerStep) {
-    const int t = tb + grp;
-    const bool valid = t < t_end;
-    uint4 kr[NV], vr[NV];
-    if (valid && t == p.slot) {
-      const __nv_bfloat16* kn = reinterpret_cast<const __nv_bfloat16*>(p.k_new) + new_off;
-      const __nv_bfloat16* vn = reinterpret_cast<const __nv_bfloat16*>(p.v_new) + new_off;
+  for (int i = 0; i < n_st && ok; ++i) {
+    const int s = i % kDecStages;
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, p.err, ERR_WAIT_TMA));
+    if (!ok) break;
+    const uint8_t* ks = dsm + PL::kOffK + s * PL::kTileBytes;
+    const uint8_t* vs = dsm + PL::kOffV + s * PL::kTileBytes;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int row = warp * 8 + pass * 4 + grp;  // row within the stage
+      const int t = t_begin + i * kDecRows + row;
+      const bool valid = t < t_end;
+      uint4 kr[NV], vr[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        kr[v] = *reinterpret_cast<const uint4*>(kn + v * 8);
-        vr[v] = *reinterpret_cast<const uint4*>(vn + v * 8);
-        *reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(kc) + t * row_elems + v * 8) = kr[v];
-        *reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(vc) + t * row_elems + v * 8) = vr[v];
+        kr[v] = *reinterpret_cast<const uint4*>(ks + row * PL::kRowBytes + v * 128 + sub * 16);
+        vr[v] = *reinterpret_cast<const uint4*>(vs + row * PL::kRowBytes + v * 128 + sub * 16);
       }
-    } else if (valid) {
+      if (valid && t == p.slot) {
+        // the new token: its K/V come from the inputs and go into the cache here
+        const __nv_bfloat16* kn = reinterpret_cast<const __nv_bfloat16*>(p.k_new) + new_off;
+        const __nv_bfloat16* vn = reinterpret_cast<const __nv_bfloat16*>(p.v_new) + new_off;
+        __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(p.k_cache) +
+                            (static_cast<int64_t>(b) * p.W + t) * row_elems + kvh * D + sub * 8;
+        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(p.v_cache) +
+                            (static_cast<int64_t>(b) * p.W + t) * row_elems + kvh * D + sub * 8;
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        kr[v] = ld_stream(kc + t * row_elems + v * 8);
-        vr[v] = ld_stream(vc + t * row_elems + v * 8);
-      }
-    } else {
-#pragma unroll
-      for (int v = 0; v < NV; ++v) kr[v] = vr[v] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    float2 kf[EL / 2], vf[EL / 2];
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const uint32_t wk[4] = {kr[v].x, kr[v].y, kr[v].z, kr[v].w};
-      const uint32_t wv[4] = {vr[v].x, vr[v].y, vr[v].z, vr[v].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        kf[v * 4 + e] = make_float2(bf_lo(wk[e]), bf_hi(wk[e]));
-        vf[v * 4 + e] = make_float2(bf_lo(wv[e]), bf_hi(wv[e]));
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < EL / 2; ++e) acc = __ffma2_rn(q[g][e], kf[e], acc);
-      float s = acc.x + acc.y;
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if (valid) {
-        if (m[g] == -INFINITY || s > m[g] + 8.f) {
-          // move the reference maximum (rare after the first rows)
-          const float corr = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - s);
-          l[g] *= corr;
-#pragma unroll
-          for (int e = 0; e < EL / 2; ++e) o[g][e] = make_float2(o[g][e].x * corr, o[g][e].y * corr);
-          m[g] = s;
+        for (int v = 0; v < NV; ++v) {
+          kr[v] = *reinterpret_cast<const uint4*>(kn + v * 64);
+          vr[v] = *reinterpret_cast<const uint4*>(vn + v * 64);
+          *reinterpret_cast<uint4*>(kc + v * 64) = kr[v];
+          *reinterpret_cast<uint4*>(vc + v * 64) = vr[v];
         }
-        const float pe = ex2_approx(s - m[g]);
-        l[g] += pe;
-        const float2 p2 = make_float2(pe, pe);
+      }
+      float2 kf[4 * NV];
 #pragma unroll
-        for (int e = 0; e < EL / 2; ++e) o[g][e] = __ffma2_rn(p2, vf[e], o[g][e]);
+      for (int v = 0; v < NV; ++v) unpack8(kr[v], &kf[4 * v]);
+      float sc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4 * NV; ++e) acc = __ffma2_rn(q[g][e], kf[e], acc);
+        float x = acc.x + acc.y;
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        sc[g] = x;
+      }
+      if (valid) {
+        float2 vf[4 * NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) unpack8(vr[v], &vf[4 * v]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (m[g] == -INFINITY || sc[g] > m[g] + 8.f) {
+            // move the reference maximum (rare after the first rows)
+            const float corr = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - sc[g]);
+            l[g] *= corr;
+#pragma unroll
+            for (int e = 0; e < 4 * NV; ++e) o[g][e] = make_float2(o[g][e].x * corr, o[g][e].y * corr);
+            m[g] = sc[g];
+          }
+          const float pe = ex2_approx(sc[g] - m[g]);
+          l[g] += pe;
+          const float2 p2 = make_float2(pe, pe);
+#pragma unroll
+          for (int e = 0; e < 4 * NV; ++e) o[g][e] = __ffma2_rn(p2, vf[e], o[g][e]);
+        }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+    if (threadIdx.x == 0 && i + kDecStages < n_st) {
+      // refill this stage once all four warps have read it
+      if (!mbar_wait(bar_empty + 8 * s, (i / kDecStages) & 1, p.err, ERR_WAIT_TMA)) ok = false;
+      else issue(i + kDecStages);
+    }
+  }
+  // never leave with a bulk copy still landing in shared memory
+  if (threadIdx.x == 0) {
+    for (int i = imax(0, n_st - kDecStages); i < n_st; ++i)
+      mbar_wait(bar_full + 8 * (i % kDecStages), (i / kDecStages) & 1, p.err, ERR_WAIT_TMA);
   }
 
   // ---- merge the four row groups of each warp with shuffles, then the four
-  // warps through shared memory
+  // warps through shared memory (reusing the first stage's K tile)
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     float M = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], 8));
@@ -158,7 +223,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeParams 
     lw += __shfl_xor_sync(0xffffffffu, lw, 8);
     lw += __shfl_xor_sync(0xffffffffu, lw, 16);
 #pragma unroll
-    for (int e = 0; e < EL / 2; ++e) {
+    for (int e = 0; e < 4 * NV; ++e) {
       float x = o[g][e].x * wgt, y = o[g][e].y * wgt;
       x += __shfl_xor_sync(0xffffffffu, x, 8);
       x += __shfl_xor_sync(0xffffffffu, x, 16);
@@ -169,20 +234,24 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeParams 
     m[g] = M;
     l[g] = lw;
   }
-  __shared__ float sm_m[4][G], sm_l[4][G];
-  __shared__ float sm_o[4][G][D];
+  __syncthreads();
+  float* sm_o = reinterpret_cast<float*>(dsm);              // [4][G][D]
+  float* sm_ml = sm_o + 4 * G * D;                          // [4][G][2]
   if (grp == 0) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (sub == 0) {
-        sm_m[warp][g] = m[g];
-        sm_l[warp][g] = l[g];
+        sm_ml[(warp * G + g) * 2] = m[g];
+        sm_ml[(warp * G + g) * 2 + 1] = l[g];
       }
 #pragma unroll
-      for (int e = 0; e < EL / 2; ++e) {
-        sm_o[warp][g][sub * EL + 2 * e] = o[g][e].x;
-        sm_o[warp][g][sub * EL + 2 * e + 1] = o[g][e].y;
-      }
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int d = 64 * v + 8 * sub + 2 * e;
+          sm_o[(warp * G + g) * D + d] = o[g][4 * v + e].x;
+          sm_o[(warp * G + g) * D + d + 1] = o[g][4 * v + e].y;
+        }
     }
   }
   __syncthreads();
@@ -191,14 +260,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeParams 
     const int g = idx / D, d = idx - g * D;
     float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) M = fmaxf(M, sm_m[r][g]);
+    for (int r = 0; r < 4; ++r) M = fmaxf(M, sm_ml[(r * G + g) * 2]);
     float L = 0.f, acc = 0.f;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float mr = sm_m[r][g];
+      const float mr = sm_ml[(r * G + g) * 2];
       const float wgt = (mr == -INFINITY) ? 0.f : ex2_approx(mr - M);
-      L += wgt * sm_l[r][g];
-      acc += wgt * sm_o[r][g][d];
+      L += wgt * sm_ml[(r * G + g) * 2 + 1];
+      acc += wgt * sm_o[(r * G + g) * D + d];
     }
     p.part_o[(part + g) * D + d] = acc;
     if (d == 0) {
@@ -259,11 +328,16 @@ __global__ void decode_write_f32_kernel(const DecodeParams p) {
 }  // namespace
 
 int decode_chunks(int B, int Hkv, int W) {
-  // enough CTAs for ~28 per SM on 148 SMs, chunks of at least 64 slots
+  // enough CTAs for ~16 per SM on 148 SMs, chunks of at least 2 pipeline stages
   const int64_t pairs = static_cast<int64_t>(B) * Hkv;
-  int chunks = static_cast<int>((148LL * 28 + pairs - 1) / pairs);
-  chunks = imax(1, imin(chunks, cdiv(W, 64)));
+  int chunks = static_cast<int>((148LL * 16 + pairs - 1) / pairs);
+  chunks = imax(1, imin(chunks, cdiv(W, 2 * kDecRows)));
   return chunks;
+}
+
+int decode_chunk_len(int n_valid, int chunks) {
+  // whole pipeline stages per chunk
+  return cdiv(cdiv(n_valid, chunks), kDecRows) * kDecRows;
 }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
@@ -273,16 +347,37 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
   return n * D * sizeof(float) + n * 2 * sizeof(float);
 }
 
-cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
-  const int G = p.Hq / p.Hkv;
-  dim3 grid(p.chunks, p.Hkv, p.B);
-#define SWA_DEC_CASE(DD, GG)                                                   \
-  if (p.D == DD && G == GG) {                                                  \
-    decode_kernel<DD, GG><<<grid, kDecThreads, 0, stream>>>(p);                \
-    decode_combine_kernel<DD><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);    \
-    count_launches(2);                                                         \
-    return cudaGetLastError();                                                 \
+namespace {
+template <int D, int G>
+cudaError_t launch_dec(const DecodeParams& p, cudaStream_t stream) {
+  static int attr_dev_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const int bit = 1 << (dev & 31);
+  if (!(attr_dev_mask & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               DecPlan<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_dev_mask |= bit;
   }
+  dim3 grid(p.chunks, p.Hkv, p.B);
+  decode_kernel<D, G><<<grid, kDecThreads, DecPlan<D>::kSmemBytes, stream>>>(p);
+  decode_combine_kernel<D><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
+  count_launches(2);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_decode_bf16(const DecodeParams& p_in, cudaStream_t stream) {
+  const int G = p_in.Hq / p_in.Hkv;
+  DecodeParams p = p_in;
+  // K/V caches viewed as rows [B*W, Hkv, D]; one box = 32 rows of one KV head
+  if (!encode_rows_map(&p.tm_k, p.k_cache, p.D, p.Hkv, static_cast<int64_t>(p.B) * p.W, kDecRows) ||
+      !encode_rows_map(&p.tm_v, p.v_cache, p.D, p.Hkv, static_cast<int64_t>(p.B) * p.W, kDecRows))
+    return cudaErrorInvalidValue;
+  p.chunk_len = decode_chunk_len(p.n_valid, p.chunks);
+#define SWA_DEC_CASE(DD, GG) \
+  if (p.D == DD && G == GG) return launch_dec<DD, GG>(p, stream);
   SWA_DEC_CASE(128, 1) SWA_DEC_CASE(128, 2) SWA_DEC_CASE(128, 4) SWA_DEC_CASE(128, 8)
   SWA_DEC_CASE(64, 1) SWA_DEC_CASE(64, 2) SWA_DEC_CASE(64, 4) SWA_DEC_CASE(64, 8)
 #undef SWA_DEC_CASE

@@ -96,7 +96,6 @@ extern "C" swa_status swa_decode_noalloc(const void* q, const void* k_new, const
   p.n_valid = (pos >= W - 1) ? W : static_cast<int>(pos + 1);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   p.chunks = swa::decode_chunks(B, Hkv, W);
-  p.chunk_len = swa::cdiv(p.n_valid, p.chunks);
   const size_t n_part = static_cast<size_t>(B) * Hkv * p.chunks * G;
   p.part_o = static_cast<float*>(scratch);
   p.part_ml = p.part_o + n_part * head_dim;

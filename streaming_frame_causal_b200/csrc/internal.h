@@ -77,6 +77,8 @@ cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
+  CUtensorMap tm_k;   // K cache as rows [B*W, Hkv, D], box = 32 rows x 1 head x D
+  CUtensorMap tm_v;
   const void* q;      // [B, Hq, D]
   const void* k_new;  // [B, Hkv, D]
   const void* v_new;
@@ -92,6 +94,9 @@ struct DecodeParams {
 };
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
+int decode_chunk_len(int n_valid, int chunks);
+// bf16 [rows, H, D] as a 3-D tensor map with a box of box_rows rows of one head (no swizzle)
+bool encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows);
 int decode_chunks(int B, int Hkv, int W);
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);
