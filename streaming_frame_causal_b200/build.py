@@ -25,6 +25,8 @@ LIB = os.path.join(PKG, "libswa_b200.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]
+# extra nvcc flags for tuning builds, e.g. SWA_NVCC_FLAGS="-DSWA_POLY_PAIRS=4"
+EXTRA = os.environ.get("SWA_NVCC_FLAGS", "").split()
 
 
 def _nvcc() -> str:
@@ -41,7 +43,7 @@ def _deps_mtime() -> float:
 
 def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [_nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [_nvcc(), *ARCH, *FLAGS, *EXTRA, "-c", src, "-o", obj]
     if ptxas_v:
         cmd += ["-Xptxas", "-v"]
     if verbose:
@@ -56,7 +58,7 @@ def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
 
 def build(verbose: bool = False, force: bool = False, ptxas_v: bool = False) -> str:
     """Compile and link the library if any source is newer than it; return its path."""
-    if not force and not ptxas_v and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
+    if not force and not ptxas_v and not EXTRA and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
