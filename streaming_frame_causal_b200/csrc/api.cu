@@ -105,7 +105,6 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B) 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int64_t imin64h(int64_t a, int64_t b) { return a < b ? a : b; }
 
 }  // namespace
 
@@ -249,12 +248,11 @@ extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, v
   p.S = Sc;
   p.Wf = Wf;
   p.n_pairs = qpairs_per_frame(P);
+  p.splits = 1;
   p.scale_log2 = scale_log2(head_dim);
   const int64_t items = static_cast<int64_t>(S) * B * heads * p.n_pairs;
   if (items > 0x7fffffffLL) return SWA_ERR_SHAPE;
-  p.n_items = static_cast<int>(items);
-  // one unit per CTA: the hardware hands out these long CTAs longest first
-  return cuda_status(launch_attn_tc(p, head_dim, static_cast<int>(items), st));
+  return cuda_status(launch_attn_tc(p, head_dim, items, st));
 }
 
 // =================================================================== band GQA
@@ -303,14 +301,13 @@ extern "C" swa_status swa_band_prefill(const void* q, const void* k, const void*
   p.Hkv = Hkv;
   p.W = window;
   p.n_qtiles = cdiv(N, kTileRows);
+  p.splits = 1;
   p.scale_log2 = scale_log2(head_dim);
   const int G = Hq / Hkv;
   const int per_group = (G % 2 == 0) ? G / 2 : G;
   const int64_t items = static_cast<int64_t>(p.n_qtiles) * B * Hkv * per_group;
   if (items > 0x7fffffffLL) return SWA_ERR_SHAPE;
-  p.n_items = static_cast<int>(items);
-  // one unit per CTA: the hardware hands out these long CTAs longest first
-  return cuda_status(launch_attn_tc(p, head_dim, static_cast<int>(items), st));
+  return cuda_status(launch_attn_tc(p, head_dim, items, st));
 }
 
 // ==================================================================== decode
@@ -434,9 +431,9 @@ bool stream_geom(const swa_stream_cfg* c, StreamGeom* g) {
   g->meta_ints = 8 + g->n_slots + g->max_pages + 2 * g->max_segs;
   g->meta_stride = round256(static_cast<size_t>(g->meta_ints) * 4);
   g->store_bytes = round256(static_cast<size_t>(g->total_rows) * g->row_bytes);
-  // split attend: max_splits partial slots of 256 query rows per (head, tile pair)
-  const size_t part_rows = static_cast<size_t>(c->max_splits) * c->heads * qpairs_per_frame(c->P) * 256;
-  g->part_bytes = round256(part_rows * c->head_dim * 4) + round256(part_rows * 2 * 4);
+  const size_t rows_h = static_cast<size_t>(c->P) * c->heads;
+  g->part_bytes = round256(static_cast<size_t>(c->max_splits) * rows_h * c->head_dim * 4) +
+                  round256(static_cast<size_t>(c->max_splits) * rows_h * 2 * 4);
   g->total = g->meta_stride * c->num_layers + 2 * g->store_bytes * c->num_layers + g->part_bytes;
   return true;
 }
@@ -487,9 +484,10 @@ extern "C" swa_status swa_stream_create(swa_stream** out, const swa_stream_cfg* 
   h->meta0 = h->base;
   h->store0 = h->base + g.meta_stride * cfg->num_layers;
   uint8_t* part = h->store0 + 2 * g.store_bytes * cfg->num_layers;
-  const size_t part_rows = static_cast<size_t>(cfg->max_splits) * cfg->heads * qpairs_per_frame(cfg->P) * 256;
+  const size_t rows_h = static_cast<size_t>(cfg->P) * cfg->heads;
   h->part_o = reinterpret_cast<float*>(part);
-  h->part_ml = reinterpret_cast<float*>(part + round256(part_rows * cfg->head_dim * 4));
+  h->part_ml = reinterpret_cast<float*>(part + round256(static_cast<size_t>(cfg->max_splits) * rows_h *
+                                                        cfg->head_dim * 4));
   h->n_frames.assign(cfg->num_layers, 0);
   if (cfg->dtype == SWA_BF16) {
     h->tm_k.resize(cfg->num_layers);
@@ -572,18 +570,21 @@ extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int
 
 namespace {
 
-// Persistent streaming attend: grid CTAs take equal contiguous shares of the
-// items x T flattened (item, key tile) space.  An item then spans at most
-// ceil(T / share) + 1 CTAs; shrink the grid until that fits the partial slots.
-int stream_grid(int items, int T, int max_units, int sms) {
-  const int64_t total = static_cast<int64_t>(items) * T;
-  int grid = static_cast<int>(total < sms ? total : sms);
-  while (grid > 1) {
-    const int64_t L = (total + grid - 1) / grid;
-    if ((T + L - 1) / L + 1 <= max_units) break;
-    --grid;
+// split count for the streaming attend: enough CTAs to cover the SMs in few
+// waves while keeping the partial traffic small
+int choose_splits(int T, int items_per_split, int max_splits, int sms) {
+  int best = 1;
+  double best_cost = 1e300;
+  for (int k = 1; k <= max_splits && k <= T; ++k) {
+    const int64_t ctas = static_cast<int64_t>(items_per_split) * k;
+    const int64_t waves = (ctas + sms - 1) / sms;
+    const double cost = static_cast<double>(waves) * cdiv(T, k) + (k > 1 ? 2.0 + 0.25 * k : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = k;
+    }
   }
-  return grid < 1 ? 1 : grid;
+  return best;
 }
 
 }  // namespace
@@ -629,7 +630,7 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
   const int T = n_ret * cdiv(c.P, kTileRows) + cdiv(n_special, kTileRows);
   const int n_pairs = qpairs_per_frame(c.P);
   const int items = c.heads * n_pairs;
-  const int grid = stream_grid(items, T, c.max_splits, num_sms());
+  const int splits = choose_splits(T, items, c.max_splits, num_sms());
   TcParams p;
   std::memset(&p, 0, sizeof(p));
   if (!make_map(&p.tm_q, q_frame, c.head_dim, c.heads, c.P, 1)) return SWA_ERR_CUDA;
@@ -649,16 +650,12 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
   p.Hkv = c.heads;
   p.P = c.P;
   p.n_pairs = n_pairs;
-  p.n_items = items;
-  p.max_units = c.max_splits;
+  p.splits = splits;
   p.max_segs = h->max_segs;
   p.scale_log2 = scale_log2(c.head_dim);
-  cudaError_t e = launch_attn_tc(p, c.head_dim, grid, st);
+  cudaError_t e = launch_attn_tc(p, c.head_dim, static_cast<int64_t>(items) * splits, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
-  // items split across CTAs need the merge; none are when every share is whole items
-  const int64_t total = static_cast<int64_t>(items) * T;
-  const int64_t L = (total + grid - 1) / grid;
-  if (L % T != 0) e = launch_stream_combine(p, c.head_dim, grid, st);
+  if (splits > 1) e = launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, c.head_dim, splits, st);
   return cuda_status(e);
 }
 

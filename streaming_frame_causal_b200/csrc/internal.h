@@ -16,8 +16,8 @@ struct TcParams {
   CUtensorMap tm_k;   // K as 4-D {D, Hkv, Nk, B}
   CUtensorMap tm_v;   // V, same shape as K
   void* out;          // bf16 [B, Nq, Hq, D] (final output)
-  float* part_o;      // f32 [n_items, max_units, 256, D] (partial numerators of split items)
-  float* part_ml;     // f32 [n_items, max_units, 256, 2] (running max in log2 units, row sum)
+  float* part_o;      // f32 [splits, Nq, Hq, D] (split-KV partial numerators)
+  float* part_ml;     // f32 [splits, Nq, Hq, 2] (running max in log2 units, row sum)
   const int* seg_row; // stream mode: key segments (storage row, length) on the device
   const int* seg_len;
   const int* meta_hdr;
@@ -26,16 +26,14 @@ struct TcParams {
   int B, Nq, Hq, Hkv;
   int P, F, S, Wf, n_pairs;  // frame mode (P, n_pairs also stream mode)
   int W, n_qtiles;           // band mode
-  int n_items;               // work items (query-tile pairs) of the launch
-  int max_units, max_segs;   // stream mode: partial slots per item, metadata capacity
+  int splits, max_segs;      // stream mode
   float scale_log2;          // log2(e) / sqrt(D)
 };
 
-// persistent launch: ``grid`` CTAs loop over the items
-cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream);
 int tc_smem_bytes(int head_dim);
-// merges the partials of streaming items that were split across CTAs
-cudaError_t launch_stream_combine(const TcParams& p, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
+                           int head_dim, int splits, cudaStream_t stream);
 
 // ---------------------------------------------------------------- SIMT f32 path
 enum SimtMode : int { SIMT_FRAME = 0, SIMT_BAND = 1, SIMT_STREAM = 2, SIMT_DECODE = 3 };
