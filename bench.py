@@ -184,6 +184,31 @@ def gpu_smi_id(torch, dev, fallback):
         return str(fallback)
 
 
+# ---------------------------------------------------------------- multi-GPU plumbing
+# The path shards into independent units (clips, streams, decode batches): every
+# rank runs its own shard of the per-GPU workload with no collective on the data
+# path (weak scaling).  Collectives appear only around the timed region: a
+# barrier on entry and exit and a max over ranks of the device-timed elapsed time.
+def shard_seed(rank: int) -> int:
+    """Seed offset of a rank's shard: ranks draw disjoint synthetic inputs."""
+    return 1000 * rank
+
+
+def max_over_ranks(elapsed_ms: float, world: int, device) -> float:
+    """Elapsed time of the slowest rank (all ranks must call it in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, work_per_rank_step: float, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * work_per_rank_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -195,7 +220,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    seed = 1000 * rank
+    seed = shard_seed(rank)
 
     # ---- inputs (synthetic, seeded; shard = this rank's independent work)
     use = (lambda s: args.stage in ("all", s))
@@ -227,7 +252,7 @@ def run_ours(args, rank, world, local_rank):
         total_frames = ST["S"] + ST["Wc"] + (args.warmup + 2 * args.steps + 4) * ST["frames_per_step"]
         cache = swa.SwaStream(num_layers=1, heads=ST["H"], head_dim=ST["D"], P=ST["P"], scale_frames=ST["S"],
                               window_frames=ST["Wc"], page_tokens=ST["page"], max_frames=total_frames,
-                              device=dev)
+                              max_splits=12, device=dev)
 
     def stream_frame(fr=None):
         i = state["frame"]
@@ -297,15 +322,12 @@ def run_ours(args, rank, world, local_rank):
             part_ms[name] += ev[s][j].elapsed_time(ev[s][j + 1])
     if swa.swa_device_error_check() != 0:
         raise RuntimeError("device error flag set during the timed region")
-    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_ms / args.steps
     stage_flops = {"prefill": flops_prefill(), "stream": ST["frames_per_step"] * flops_stream_frame(),
                    "band": flops_band(), "decode": flops_decode()}
     flops = sum(stage_flops[n] for n, _ in parts)
-    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops, args.steps, elapsed_ms)
 
     peaks = measured_peaks()
     per = {k: v / args.steps for k, v in part_ms.items()}
@@ -421,11 +443,8 @@ def run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk, bv, 
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": world * flops * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    ms = max_over_ranks(ms, world, dev)
+    return {"value": weak_scaling_value(world, flops, steps, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": ms / steps}
 

@@ -129,7 +129,7 @@ typedef struct swa_stream_cfg {
     int num_special;         /* camera + register tokens at the head of every frame     */
     int max_frames;          /* frames per layer the buffer is sized for               */
     int dtype;               /* swa_dtype of K/V/Q/out                                  */
-    int max_splits;          /* split-KV partial buffers for the attend (>= 1)          */
+    int max_splits;          /* split-KV partial buffers for the attend (1..32)         */
 } swa_stream_cfg;
 
 typedef struct swa_stream swa_stream;  /* opaque host handle */

@@ -244,7 +244,7 @@ class SwaStream:
 
     def __init__(self, num_layers: int, heads: int, head_dim: int, P: int, scale_frames: int,
                  window_frames: int, page_tokens: int = 16, cross_frame_special: bool = False,
-                 num_special: int = 5, max_frames: int = 1024, dtype=torch.bfloat16, max_splits: int = 16,
+                 num_special: int = 5, max_frames: int = 1024, dtype=torch.bfloat16, max_splits: int = 12,
                  device="cuda", stream=None):
         self.cfg = _make_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_tokens,
                              cross_frame_special, num_special, max_frames, dtype, max_splits)

@@ -412,7 +412,7 @@ bool stream_geom(const swa_stream_cfg* c, StreamGeom* g) {
   if (!c) return false;
   if (c->num_layers < 1 || c->heads < 1 || c->head_dim < 1 || c->P < 1 || c->scale_frames < 0 ||
       c->page_tokens < 1 || c->num_special < 0 || c->num_special > c->P || c->max_frames < 1 ||
-      c->max_splits < 1 || (c->dtype != SWA_F32 && c->dtype != SWA_BF16))
+      c->max_splits < 1 || c->max_splits > 32 || (c->dtype != SWA_F32 && c->dtype != SWA_BF16))
     return false;
   const int esize = c->dtype == SWA_F32 ? 4 : 2;
   g->row_bytes = c->heads * c->head_dim * esize;

@@ -563,7 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
 // ---------------------------------------------------------------- combine
 // O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c  (m in log2 units), the
-// log-sum-exp merge of split-KV partials.  One warp per (row, head).
+// log-sum-exp merge of split-KV partials.  One warp per (row, head): lane c
+// holds split c's (m, l), the warp reduces M and the weighted sum, then every
+// lane accumulates its slice of O over the splits with independent loads.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml,
@@ -573,25 +575,48 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int lane = threadIdx.x & 31;
   if (gw >= rows * H) return;
   const int64_t stride = static_cast<int64_t>(rows) * H;
-  float M = -INFINITY;
-  for (int c = 0; c < splits; ++c) M = fmaxf(M, part_ml[(c * stride + gw) * 2]);
-  constexpr int E = D / 32;
+  float mc = -INFINITY, lc = 0.f;
+  if (lane < splits) {
+    const float2 ml = *reinterpret_cast<const float2*>(part_ml + (lane * stride + gw) * 2);
+    mc = ml.x;
+    lc = ml.y;
+  }
+  float M = mc;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float wc = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+  float L = wc * lc;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  constexpr int E = D / 32;  // elements per lane: 2 (D = 64) or 4 (D = 128)
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float L = 0.f;
   for (int c = 0; c < splits; ++c) {
-    const float mc = part_ml[(c * stride + gw) * 2];
-    if (mc == -INFINITY) continue;
-    const float wgt = exp2f(mc - M);
-    L += wgt * part_ml[(c * stride + gw) * 2 + 1];
-    const float* src = part_o + (c * stride + gw) * D;
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] += wgt * src[lane + 32 * e];
+    const float w = __shfl_sync(0xffffffffu, wc, c);
+    const float* src = part_o + (c * stride + gw) * D + lane * E;
+    if constexpr (E == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+    } else {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    }
   }
   const float inv = 1.f / L;
-#pragma unroll
-  for (int e = 0; e < E; ++e) out[static_cast<int64_t>(gw) * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+  __nv_bfloat16* dst = out + static_cast<int64_t>(gw) * D + lane * E;
+  if constexpr (E == 2) {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  } else {
+    uint2 v;
+    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = v;
+  }
 }
 
 }  // namespace
