@@ -102,9 +102,17 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_sha():
+KERNEL_SOURCES = {
+    "attn": ("attn_tc.cu", "ptx.cuh", "tile_sched.h", "exp2_poly.cuh"),
+    "decode": ("decode.cu", "ptx.cuh"),
+}
+
+
+def kernel_source_sha(kind="attn"):
+    """Hash of the sources a kernel is built from: a recorded ncu traffic figure
+    only applies while it matches."""
     h = hashlib.sha256()
-    for name in ("attn_tc.cu", "ptx.cuh", "tile_sched.h"):
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "streaming_frame_causal_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -119,7 +127,8 @@ def recorded_traffic(kernel_key):
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    kind = "decode" if kernel_key.startswith("decode") else "attn"
+    if not e or e.get("source_sha") != kernel_source_sha(kind):
         return None
     return e.get("bytes_per_launch")
 
