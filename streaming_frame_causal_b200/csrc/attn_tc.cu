@@ -9,9 +9,10 @@
 // the cache; sliding-window explainer: token band t-W+1..t).
 //
 // CTA organisation (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer: Q tiles once, then K/V key tiles into a ring
+//   warp 0      TMA producer: Q tiles once, then K key tiles into a ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 2-3   idle
+//   warp 2      idle
+//   warp 3      TMA producer: V key tiles into a second ring
 //   warps 4-7   softmax for query tile A (one thread per query row)
 //   warps 8-11  softmax for query tile B
 // After set-up, warpgroup 0 gives registers back (setmaxnreg.dec to 64) and the
@@ -69,7 +70,7 @@ struct Plan {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 2;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
 };
@@ -231,27 +232,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // barriers
   const uint32_t bar0 = base + PL::kOffBar;
   auto q_full = [&](int g) { return bar0 + 8u * g; };
-  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + PL::kStages + s); };
-  auto s_full = [&](int g) { return bar0 + 8u * (2 + 2 * PL::kStages + g); };
-  auto p_full = [&](int g) { return bar0 + 8u * (4 + 2 * PL::kStages + g); };
-  const uint32_t o_full = bar0 + 8u * (6 + 2 * PL::kStages);
-  const uint32_t drain = bar0 + 8u * (7 + 2 * PL::kStages);
+  // K and V stages have their own barriers: K_j is released once both tiles'
+  // QK^T(j) are issued, V_j once both PV(j) are, so the K ring runs ahead
+  auto k_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (2 + PL::kStages + s); };
+  auto k_empty = [&](int s) { return bar0 + 8u * (2 + 2 * PL::kStages + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (2 + 3 * PL::kStages + s); };
+  constexpr int kB = 2 + 4 * PL::kStages;
+  auto s_full = [&](int g) { return bar0 + 8u * (kB + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (kB + 2 + g); };
+  auto o_full = [&](int g) { return bar0 + 8u * (kB + 4 + g); };
+  auto drain = [&](int g) { return bar0 + 8u * (kB + 6 + g); };
   const uint32_t tmem_slot = base + PL::kOffTmem;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full(0), 1);
     mbar_init(q_full(1), 1);
     for (int s = 0; s < PL::kStages; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_empty(s), 1);
     }
     mbar_init(s_full(0), 1);
     mbar_init(s_full(1), 1);
     mbar_init(p_full(0), 128);
     mbar_init(p_full(1), 128);
-    mbar_init(o_full, 1);
-    mbar_init(drain, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(o_full(g), 1);
+      mbar_init(drain(g), 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -264,26 +274,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + PL::kOffTmem);
   if (warp < 4) {
   reg_dealloc<kRegsCtl>();
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers
+    // lane 0 of warp 0 loads the Q tiles and the K ring, lane 0 of warp 3 the V ring
+    const bool is_k = (warp == 0);
     if (lane == 0 && T > 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      for (int g = 0; g < (has_b ? 2 : 1); ++g) {
-        mbar_arrive_expect_tx(q_full(g), PL::kTileBytes);
-        for (int sub = 0; sub < PL::kSubs; ++sub)
-          tma_load_4d(base + PL::kOffQ + g * PL::kTileBytes + sub * kSubBytes, &p.tm_q, q_full(g),
-                      sub * 64, g ? w.h1 : w.h0, g ? w.qrow1 : w.qrow0, w.b);
+      const CUtensorMap* tm = is_k ? &p.tm_k : &p.tm_v;
+      tma_prefetch_desc(tm);
+      if (is_k) {
+        tma_prefetch_desc(&p.tm_q);
+        for (int g = 0; g < (has_b ? 2 : 1); ++g) {
+          mbar_arrive_expect_tx(q_full(g), PL::kTileBytes);
+          for (int sub = 0; sub < PL::kSubs; ++sub)
+            tma_load_4d(base + PL::kOffQ + g * PL::kTileBytes + sub * kSubBytes, &p.tm_q, q_full(g),
+                        sub * 64, g ? w.h1 : w.h0, g ? w.qrow1 : w.qrow0, w.b);
+        }
       }
+      const uint32_t ring = base + (is_k ? PL::kOffK : PL::kOffV);
       Cursor cur;
       bool ok = cursor_seek(w, w.t_begin, cur);
       if (!ok) atomicOr(p.err, ERR_BAD_META);
       int issued = 0;
       for (int j = 0; j < T && ok; ++j) {
         const int st = j % PL::kStages;
-        if (j >= PL::kStages &&
-            !mbar_wait(kv_empty(st), ((j / PL::kStages) - 1) & 1, p.err, ERR_WAIT_TMA)) {
+        const uint32_t full = is_k ? k_full(st) : v_full(st);
+        if (j >= PL::kStages && !mbar_wait(is_k ? k_empty(st) : v_empty(st), ((j / PL::kStages) - 1) & 1,
+                                           p.err, ERR_WAIT_TMA)) {
           ok = false;
           break;
         }
@@ -294,50 +310,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         int krow, kvalid;
         cursor_tile(w, cur, &krow, &kvalid);
-        mbar_arrive_expect_tx(kv_full(st), 2 * PL::kTileBytes);
-        for (int sub = 0; sub < PL::kSubs; ++sub) {
-          tma_load_4d(base + PL::kOffK + st * PL::kTileBytes + sub * kSubBytes, &p.tm_k,
-                      kv_full(st), sub * 64, w.kvh, krow, w.b);
-          tma_load_4d(base + PL::kOffV + st * PL::kTileBytes + sub * kSubBytes, &p.tm_v,
-                      kv_full(st), sub * 64, w.kvh, krow, w.b);
-        }
+        mbar_arrive_expect_tx(full, PL::kTileBytes);
+        for (int sub = 0; sub < PL::kSubs; ++sub)
+          tma_load_4d(ring + st * PL::kTileBytes + sub * kSubBytes, tm, full, sub * 64, w.kvh, krow, w.b);
         cursor_next(w, cur);
         ++issued;
       }
       // drain: never leave the CTA with a bulk copy still writing its shared memory
       for (int j = issued - PL::kStages; j < issued; ++j) {
         if (j < 0) continue;
-        mbar_wait(kv_full(j % PL::kStages), (j / PL::kStages) & 1, p.err, ERR_WAIT_TMA);
+        mbar_wait(is_k ? k_full(j % PL::kStages) : v_full(j % PL::kStages), (j / PL::kStages) & 1, p.err,
+                  ERR_WAIT_TMA);
       }
-      for (int g = 0; g < (has_b ? 2 : 1); ++g) mbar_wait(q_full(g), 0, p.err, ERR_WAIT_TMA);
+      if (is_k)
+        for (int g = 0; g < (has_b ? 2 : 1); ++g) mbar_wait(q_full(g), 0, p.err, ERR_WAIT_TMA);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Lane 0 issues every tcgen05.mma.  The issue path is kept short (a
+    // single thread's instruction latency bounds the MMA rate for N <= 128):
+    // shared-memory descriptors are built once, and a K step or a ring stage
+    // moves the start-address field by a constant (addresses stay below 2^18,
+    // so the 14-bit field never carries).
     if (lane == 0 && T > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
+      constexpr uint64_t kStageStep = PL::kTileBytes >> 4;
+      const uint64_t dq0 = sdesc_sw128(base + PL::kOffQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(base + PL::kOffK, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(base + PL::kOffV, kSubBytes, 1024);
       auto issue_qk = [&](int g, int st) {
-        const uint32_t qa = base + PL::kOffQ + g * PL::kTileBytes;
-        const uint32_t kb = base + PL::kOffK + st * PL::kTileBytes;
+        const uint64_t dq = dq0 + g * kStageStep;  // Q tiles are kTileBytes apart too
+        const uint64_t dk = dk0 + st * kStageStep;
+        const uint32_t tS = tmem + PL::col_s(g);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-          mma_ss(tmem + PL::col_s(g), sdesc_sw128(qa + off, 16, 1024),
-                 sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kSubBytes + (kk & 3) * 32) >> 4);
+          mma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int g, int st, bool acc) {
-        const uint32_t vb = base + PL::kOffV + st * PL::kTileBytes;
+        const uint64_t dv = dv0 + st * kStageStep;
+        const uint32_t tP = tmem + PL::col_p(g), tO = tmem + PL::col_o(g);
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          mma_ts(tmem + PL::col_o(g), tmem + PL::col_p(g) + kk * 8,
-                 sdesc_sw128(vb + kk * 16 * 128, kSubBytes, 1024), idesc_pv,
-                 (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          mma_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(q_full(0), 0, p.err, ERR_WAIT_MMA);
       if (ok && has_b) ok = mbar_wait(q_full(1), 0, p.err, ERR_WAIT_MMA);
-      if (ok) ok = mbar_wait(kv_full(0), 0, p.err, ERR_WAIT_MMA);
+      if (ok) ok = mbar_wait(k_full(0), 0, p.err, ERR_WAIT_MMA);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -346,35 +367,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           issue_qk(1, 0);
           mma_commit(s_full(1));
         }
+        mma_commit(k_empty(0));
       }
+      const int ng = has_b ? 2 : 1;
+      // Fixed order per key tile: PV_A(j) QK_A(j+1) | PV_B(j) QK_B(j+1), each
+      // tile's MMAs back to back with its commit after them.  At head_dim 128
+      // P_g aliases S_g: QK_g(j+1) follows PV_g(j) in this thread's issue
+      // order, which the tensor core keeps.
       for (int j = 0; j < T && ok; ++j) {
         const int st = j % PL::kStages;
         const int st1 = (j + 1) % PL::kStages;
         const bool more = j + 1 < T;
-        if (!mbar_wait(p_full(0), j & 1, p.err, ERR_WAIT_MMA)) break;
-        tc_fence_after();
-        issue_pv(0, st, j > 0);
-        if (more) {
-          if (!mbar_wait(kv_full(st1), ((j + 1) / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+        if (more && !mbar_wait(k_full(st1), ((j + 1) / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+        if (!mbar_wait(v_full(st), (j / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g) {
+          if (!mbar_wait(p_full(g), j & 1, p.err, ERR_WAIT_MMA)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          issue_qk(0, st1);
-          mma_commit(s_full(0));
+          issue_pv(g, st, j > 0);
+          if (more) {
+            issue_qk(g, st1);
+            mma_commit(s_full(g));
+          } else {
+            mma_commit(o_full(g));
+          }
         }
-        if (has_b) {
-          if (!mbar_wait(p_full(1), j & 1, p.err, ERR_WAIT_MMA)) break;
-          tc_fence_after();
-          issue_pv(1, st, j > 0);
-        }
-        mma_commit(kv_empty(st));
-        if (has_b && more) {
-          issue_qk(1, st1);
-          mma_commit(s_full(1));
-        }
-        if (!more) mma_commit(o_full);
+        if (!ok) break;
+        mma_commit(v_empty(st));
+        if (more) mma_commit(k_empty(st1));
       }
       // drain every MMA this thread issued before the CTA may free TMEM
-      mma_commit(drain);
-      mbar_wait(drain, 0, p.err, ERR_WAIT_MMA);
+      mma_commit(drain(0));
+      mbar_wait(drain(0), 0, p.err, ERR_WAIT_MMA);
     }
   }
   } else {
@@ -504,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     // ---- epilogue
     if (active && ok) {
-      if (__all_sync(0xffffffffu, mbar_wait(o_full, 0, p.err, ERR_WAIT_EPI))) {
+      if (__all_sync(0xffffffffu, mbar_wait(o_full(g), 0, p.err, ERR_WAIT_EPI))) {
         tc_fence_after();
         const bool store = r < my_rows;
         const int row = my_row0 + r;
