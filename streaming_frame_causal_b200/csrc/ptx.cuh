@@ -63,19 +63,6 @@ SWA_DEV bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 // Wait for the phase with the given parity to complete.  Gives up when the
 // deadline passes or when another thread has already latched an error; on
 // giving up it latches ``code`` and returns false.
-// non-blocking probe: has the phase with this parity completed?
-SWA_DEV bool mbar_test(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 SWA_DEV bool mbar_wait(uint32_t addr, uint32_t parity, int* err, int code) {
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = global_timer_ns();

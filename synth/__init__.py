@@ -111,3 +111,38 @@ def decode_inputs(seed: int = 1, B: int = 64, W: int = 4096, Hq: int = 32, Hkv: 
     k_new = torch.randn(B, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
     v_new = torch.randn(B, Hkv, D, generator=g, dtype=torch.float32).to(dtype)
     return q, k_new, v_new, k_cache, v_cache
+
+
+def growing_scores_qkv(seed: int = 7, P: int = 1000, H: int = 2, D: int = 64, steps=None,
+                       q_scale: float = 4.0, noise: float = 0.05, dtype=torch.bfloat16):
+    """One frame of P tokens whose key tiles (128 keys each) carry a rising common
+    component, so a query row's largest score moves up from key tile to key tile.
+
+    Every query row is ``q_scale`` times the all-ones vector, with the sign
+    alternating between rows (even rows +, odd rows -).  Key rows are
+    ``beta[t] / sqrt(D)`` times the all-ones vector plus ``noise`` times a normal
+    draw, where t is the key's 128-token tile and ``beta`` the running sum of
+    ``steps`` (default: eleven steps of 10 and one of 100, in units of
+    log2(e)-scaled scores, converted here to raw values).  Values are normal.
+    The tensors are [1, P, H, D].
+    """
+    if steps is None:
+        steps = [10.0] * 5 + [100.0] + [10.0] * 6
+    g = _gen(seed)
+    # raw score of a +row against tile t is q_scale * sqrt(D) * beta[t]; choose beta so
+    # that score * log2(e) / sqrt(D) rises by steps[t] from tile t-1 to tile t
+    log2e = 1.4426950408889634
+    unit = q_scale * log2e  # log2-scaled score per unit of beta
+    beta = []
+    acc = 0.0
+    n_tiles = (P + 127) // 128
+    for t in range(n_tiles):
+        if t > 0:
+            acc += steps[(t - 1) % len(steps)] / unit
+        beta.append(acc)
+    sign = torch.where(torch.arange(P) % 2 == 0, 1.0, -1.0).view(1, P, 1, 1)
+    q = (q_scale * sign * torch.ones(1, P, H, D))
+    tile_beta = torch.tensor([beta[i // 128] for i in range(P)], dtype=torch.float32).view(1, P, 1, 1)
+    k = tile_beta / (D ** 0.5) * torch.ones(1, P, H, D) + noise * torch.randn(1, P, H, D, generator=g)
+    v = torch.randn(1, P, H, D, generator=g)
+    return q.to(dtype), k.to(dtype), v.to(dtype)

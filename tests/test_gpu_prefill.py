@@ -55,6 +55,17 @@ def test_bf16_parity_small(swa, F, P, H, sws, S, nfpb):
     check_bf16(got, _ref(q, k, v, P, S, sws, nfpb), f"bf16 F{F} P{P}")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_bf16_growing_scores(swa, D):
+    """Row maxima that climb by ~2^10 from key tile to key tile, with one jump of
+    ~2^100, on alternate rows only: exercises the rescale of O and the row sum
+    when the running max grows, the exact re-run of a tile whose scores jump too
+    far, and warps whose lanes take different branches."""
+    q, k, v = synth.growing_scores_qkv(D=D)
+    got = _run(swa, q, k, v, 1, 1000, -1, 0)
+    check_bf16(got, _ref(q, k, v, 1000, 0, -1), f"growing scores D{D}")
+
+
 def test_bf16_head_dim_128(swa):
     q, k, v = synth.tiny_qkv(seed=128, F=5, P=260, H=2, D=128, dtype=torch.bfloat16)
     got = _run(swa, q, k, v, 5, 260, 2, 1)
