@@ -25,7 +25,7 @@ LIB = os.path.join(PKG, "libswa_b200.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]
-# extra nvcc flags for tuning builds, e.g. SWA_NVCC_FLAGS="-DSWA_POLY_PAIRS=4"
+# extra nvcc flags for tuning builds, e.g. SWA_NVCC_FLAGS="-DSWA_POLY_PAIRS_D64=4"
 EXTRA = os.environ.get("SWA_NVCC_FLAGS", "").split()
 
 

@@ -56,20 +56,27 @@ struct Plan {
   static constexpr int kSubs = D / 64;                 // 64-column sub-tiles per row
   static constexpr int kTileBytes = kRows * D * 2;     // Q, K or V tile
   static constexpr int kStages = (D == 64) ? 4 : 2;    // K/V ring depth
-  // Tensor-memory columns.  D = 64: S 2x128 | P 2x64 | O 2x64.  D = 128: S 2x128 |
-  // O 2x128, and P (64 columns of bf16 pairs) reuses the first half of its own
-  // S once the softmax has read S: the next QK^T that overwrites S is issued by
-  // the same thread after the PV that reads P, and tcgen05.mma operations from
-  // one thread execute in issue order.
+  // Row sums at D = 64 come out of the PV product: V is extended by a constant
+  // 64-column block whose first column is 1, so O column D accumulates sum_k P
+  // (in f32, from the same bf16 P the PV uses) and is rescaled with O.  The PV
+  // then has N = D + 16.  At D = 128 that would not fit tensor memory; the
+  // softmax threads add the row sums themselves.
+  static constexpr bool kSumCol = (D == 64);
+  static constexpr int kON = kSumCol ? D + 16 : D;  // O columns written by the PV
+  // Tensor-memory columns: S 2x128 | O 2x128 (D or D + 16 used).  P (64 columns
+  // of bf16 pairs) reuses the first half of its own S once the softmax has read
+  // S: the next QK^T that overwrites S is issued by the same thread after the PV
+  // that reads P, and tcgen05.mma operations from one thread execute in issue order.
   SWA_DEV static uint32_t col_s(int g) { return g ? 128u : 0u; }
-  SWA_DEV static uint32_t col_p(int g) { return D == 64 ? (g ? 320u : 256u) : col_s(g); }
-  SWA_DEV static uint32_t col_o(int g) { return D == 64 ? (g ? 448u : 384u) : (g ? 384u : 256u); }
+  SWA_DEV static uint32_t col_p(int g) { return col_s(g); }
+  SWA_DEV static uint32_t col_o(int g) { return g ? 384u : 256u; }
   static constexpr uint32_t kTmemCols = 512;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffOnes = kOffV + kStages * kTileBytes;  // the constant block (kSumCol)
+  static constexpr int kOffBar = kOffOnes + (kSumCol ? kSubBytes : 0);
   static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 2;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
@@ -197,16 +204,20 @@ SWA_DEV Work decode_work(const TcParams& p) {
 }
 
 // How the 64 exponential pairs of a 128-column row are split (per group of 8 pairs):
-// the first SWA_POLY_PAIRS take 2^x on the FMA pipe (polynomial), the next
-// SWA_F16_PAIRS take one f16x2 MUFU exp2 for the pair, the rest two f32 MUFU exp2.
-// Measured on B200: 2 / 0 is fastest for head_dim 64 and close to it at 128.
-#ifndef SWA_POLY_PAIRS
-#define SWA_POLY_PAIRS 2
+// the first kPolyPairs take 2^x on the FMA pipe (polynomial), the rest two f32
+// MUFU exp2 (packed f16x2/bf16x2 MUFU exp2 yields no more results per clock).
+// Measured on B200 (same-box sweeps of 2, 3, 4): 3 is fastest at head_dim 64,
+// where the row sums come from the tensor core and leave the FMA pipe room, and
+// 2 at head_dim 128.  SWA_POLY_PAIRS_D64 / _D128 override them for tuning builds.
+#ifndef SWA_POLY_PAIRS_D64
+#define SWA_POLY_PAIRS_D64 3
 #endif
-#ifndef SWA_F16_PAIRS
-#define SWA_F16_PAIRS 0
+#ifndef SWA_POLY_PAIRS_D128
+#define SWA_POLY_PAIRS_D128 2
 #endif
-static_assert(SWA_POLY_PAIRS + SWA_F16_PAIRS <= 8, "exp2 split");
+template <int D>
+constexpr int kPolyPairs = (D == 64) ? SWA_POLY_PAIRS_D64 : SWA_POLY_PAIRS_D128;
+static_assert(SWA_POLY_PAIRS_D64 <= 8 && SWA_POLY_PAIRS_D128 <= 8, "exp2 split");
 
 SWA_DEV float max3f(float a, float b, float c) {
   float d;
@@ -267,6 +278,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (warp == 1) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
+  }
+  if constexpr (PL::kSumCol) {
+    // 128 keys x 64 columns of bf16 in the 128-byte-swizzled layout of a V
+    // sub-tile: column 0 (logical 16-byte chunk 0 of key row k, stored at
+    // physical chunk k mod 8) is 1.0, everything else 0
+    uint4* ones = reinterpret_cast<uint4*>(gbase + PL::kOffOnes);
+    for (int i = threadIdx.x; i < kSubBytes / 16; i += kThreads) {
+      const int key = i >> 3, chunk = i & 7;
+      ones[i] = make_uint4(chunk == (key & 7) ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -334,11 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // so the 14-bit field never carries).
     if (lane == 0 && T > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, PL::kON, 1);
       constexpr uint64_t kStageStep = PL::kTileBytes >> 4;
       const uint64_t dq0 = sdesc_sw128(base + PL::kOffQ, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(base + PL::kOffK, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(base + PL::kOffV, kSubBytes, 1024);
+      const uint64_t dv0 = sdesc_sw128(base + PL::kOffV, PL::kSumCol ? PL::kOffOnes - PL::kOffV : kSubBytes, 1024);
       auto issue_qk = [&](int g, int st) {
         const uint64_t dq = dq0 + g * kStageStep;  // Q tiles are kTileBytes apart too
         const uint64_t dk = dk0 + st * kStageStep;
@@ -350,7 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       };
       auto issue_pv = [&](int g, int st, bool acc) {
-        const uint64_t dv = dv0 + st * kStageStep;
+        // kSumCol: the second 64-column block of B is the ones block, at a
+        // leading-byte offset that shrinks as the stage moves up
+        const uint64_t dv = PL::kSumCol ? dv0 + st * kStageStep - ((st * kStageStep) << 16)
+                                        : dv0 + st * kStageStep;
         const uint32_t tP = tmem + PL::col_p(g), tO = tmem + PL::col_o(g);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
@@ -496,11 +521,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
           tmem_st32(tO + c0, orr);
         }
+        if constexpr (PL::kSumCol) {
+          uint32_t o16[16];
+          tmem_ld16(tO + D, o16);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) o16[c] = __float_as_uint(__uint_as_float(o16[c]) * alpha);
+          tmem_st16(tO + D, o16);
+        }
         tmem_wait_st();
       }
       l *= alpha;
       // ---- P = 2^(s*scale - m*scale): MUFU for most column pairs, the
-      // polynomial on the FMA pipe for SWA_POLY_PAIRS of every 8; packed bf16
+      // polynomial on the FMA pipe for kPolyPairs of every 8; packed bf16
       // pairs overwrite the front of s (pair pi reads s[2pi], s[2pi+1] >= pi)
       const float nb = (m == -INFINITY) ? 0.f : -m * sl2;
       const float2 c2 = make_float2(sl2, sl2);
@@ -513,16 +546,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float2 x =
             __ffma2_rn(make_float2(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])), c2, nb2);
         float2 pr;
-        if ((pi & 7) < SWA_POLY_PAIRS) {
+        if ((pi & 7) < kPolyPairs<D>) {
           pr = exp2_poly2(x);
         } else {
           pr.x = ex2_approx(x.x);
           pr.y = ex2_approx(x.y);
         }
-        acc[pi & 3] = __fadd2_rn(acc[pi & 3], pr);
+        if constexpr (!PL::kSumCol) acc[pi & 3] = __fadd2_rn(acc[pi & 3], pr);
         s[pi] = pack_bf16x2(pr.x, pr.y);
       }
-      l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+      if constexpr (!PL::kSumCol)
+        l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
       tmem_st32(tP + 0, s);
       tmem_st32(tP + 32, s + 32);
       tmem_wait_st();
@@ -533,6 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (active && ok) {
       if (__all_sync(0xffffffffu, mbar_wait(o_full(g), 0, p.err, ERR_WAIT_EPI))) {
         tc_fence_after();
+        if constexpr (PL::kSumCol) {
+          uint32_t o16[16];
+          tmem_ld16(tO + D, o16);
+          tmem_wait_ld();
+          l = __uint_as_float(o16[0]);
+        }
         const bool store = r < my_rows;
         const int row = my_row0 + r;
         const float inv = 1.f / l;
