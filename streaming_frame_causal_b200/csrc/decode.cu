@@ -6,10 +6,10 @@
 //
 // Memory-bound: every K/V byte of the buffer is read once.  Grid (chunk, kv
 // head, batch); a CTA streams one chunk of slots of one (batch, kv head) and
-// serves all G query heads of the group from the same loaded rows.  Eight lanes
-// cooperate on one cached row (16-byte vector loads, each lane a contiguous
-// slice of head_dim), so a warp covers four rows per step with fully used
-// 256-byte segments.  Scores use the scale folded into q (log2 units) and an
+// serves all G query heads of the group from the same loaded rows.  At head_dim
+// 128, sixteen lanes cooperate on one cached row (one 16-byte chunk of q, K, V
+// and O per lane and head), so a thread needs ~114 registers and four CTAs (16
+// warps) fit an SM; at head_dim 64 eight lanes share a row.  Scores use the scale folded into q (log2 units) and an
 // online softmax whose reference maximum only moves when a score exceeds it by
 // more than 2^8, so the accumulators are rarely rescaled.  Per-chunk partials
 // (max, sum, numerator) are merged by a second small kernel.
@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 
 #include <cuda.h>
 
@@ -30,9 +31,8 @@
 namespace swa {
 namespace {
 
-constexpr int kDecThreads = 128;  // 4 warps; each warp covers 4 rows per pass (8 lanes per row)
+constexpr int kDecThreads = 128;  // 4 warps
 constexpr int kDecRows = 32;      // cache rows per pipeline stage
-constexpr int kDecStages = 4;     // stages in flight per CTA
 
 SWA_DEV float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 SWA_DEV float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
@@ -52,28 +52,39 @@ SWA_DEV void tma_load_3d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, 
       : "memory");
 }
 
-template <int D>
+// LPR lanes share a cached row; ST stages of kDecRows rows are in flight per CTA.
+template <int D, int LPR, int ST>
 struct DecPlan {
+  static_assert(LPR == 8 || LPR == 16, "8 or 16 lanes per row");
+  static_assert(D % (8 * LPR) == 0, "whole 16-byte chunks per lane");
+  static constexpr int kNV = D / (8 * LPR);  // 16-byte chunks per lane per row
+  static constexpr int kRPW = 32 / LPR;      // rows a warp covers per pass
+  static constexpr int kPasses = kDecRows / (4 * kRPW);
   static constexpr int kRowBytes = D * 2;
   static constexpr int kTileBytes = kDecRows * kRowBytes;  // K (or V) rows of one stage
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kDecStages * kTileBytes;
-  static constexpr int kOffBar = 2 * kDecStages * kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 128;
+  static constexpr int kOffV = ST * kTileBytes;
+  static constexpr int kOffBar = 2 * ST * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 2 * ST * 8 + 128;
+  // CTAs per SM the launch bounds ask for (registers for 16 warps per SM when a
+  // lane holds one chunk of q and O per head)
+  static constexpr int kMinBlocks = (LPR == 16) ? 4 : 1;
 };
 
-// Lane (grp, sub) of a warp handles row grp of each 4-row pass and owns head_dim
-// elements [64v + 8 sub, 64v + 8 sub + 8) for v < D/64: its 16-byte reads of a
-// row then hit 8 distinct bank quads, so a warp's read of 4 rows takes the
-// minimum 4 shared-memory wavefronts.
-template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
-  using PL = DecPlan<D>;
-  constexpr int NV = D / 64;  // 16-byte chunks per lane per row
+// Lane (grp, sub) of a warp handles row grp of each pass and owns the head_dim
+// elements of chunks sub + LPR v (v < kNV), i.e. [8 (sub + LPR v), +8): its
+// 16-byte reads of a row hit distinct bank quads, so a warp's read of its rows
+// takes the minimum number of shared-memory wavefronts.
+template <int D, int G, int LPR, int ST>
+__global__ void __launch_bounds__(kDecThreads, DecPlan<D, LPR, ST>::kMinBlocks)
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+  using PL = DecPlan<D, LPR, ST>;
+  constexpr int NV = PL::kNV;
+  constexpr int kDecStages = ST;
   extern __shared__ __align__(128) uint8_t dsm[];
   const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane >> 3, sub = lane & 7;
+  const int grp = lane / LPR, sub = lane % LPR;
   const int t_begin = c * p.chunk_len;
   const int t_end = imin(t_begin + p.chunk_len, p.n_valid);
   const int n_st = t_end > t_begin ? cdiv(t_end - t_begin, kDecRows) : 0;
@@ -109,7 +120,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     const __nv_bfloat16* qp = qb + (static_cast<int64_t>(b) * p.Hq + kvh * G + g) * D + sub * 8;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-      unpack8(*reinterpret_cast<const uint4*>(qp + v * 64), &q[g][4 * v]);
+      unpack8(*reinterpret_cast<const uint4*>(qp + v * 8 * LPR), &q[g][4 * v]);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         q[g][4 * v + e] = make_float2(q[g][4 * v + e].x * p.scale_log2, q[g][4 * v + e].y * p.scale_log2);
@@ -135,15 +146,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     const uint8_t* ks = dsm + PL::kOffK + s * PL::kTileBytes;
     const uint8_t* vs = dsm + PL::kOffV + s * PL::kTileBytes;
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int row = warp * 8 + pass * 4 + grp;  // row within the stage
+    for (int pass = 0; pass < PL::kPasses; ++pass) {
+      const int row = (warp * PL::kPasses + pass) * PL::kRPW + grp;  // row within the stage
       const int t = t_begin + i * kDecRows + row;
       const bool valid = t < t_end;
       uint4 kr[NV], vr[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        kr[v] = *reinterpret_cast<const uint4*>(ks + row * PL::kRowBytes + v * 128 + sub * 16);
-        vr[v] = *reinterpret_cast<const uint4*>(vs + row * PL::kRowBytes + v * 128 + sub * 16);
+        kr[v] = *reinterpret_cast<const uint4*>(ks + row * PL::kRowBytes + v * 16 * LPR + sub * 16);
+        vr[v] = *reinterpret_cast<const uint4*>(vs + row * PL::kRowBytes + v * 16 * LPR + sub * 16);
       }
       if (valid && t == p.slot) {
         // the new token: its K/V come from the inputs and go into the cache here
@@ -155,10 +166,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
                             (static_cast<int64_t>(b) * p.W + t) * row_elems + kvh * D + sub * 8;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          kr[v] = *reinterpret_cast<const uint4*>(kn + v * 64);
-          vr[v] = *reinterpret_cast<const uint4*>(vn + v * 64);
-          *reinterpret_cast<uint4*>(kc + v * 64) = kr[v];
-          *reinterpret_cast<uint4*>(vc + v * 64) = vr[v];
+          kr[v] = *reinterpret_cast<const uint4*>(kn + v * 8 * LPR);
+          vr[v] = *reinterpret_cast<const uint4*>(vn + v * 8 * LPR);
+          *reinterpret_cast<uint4*>(kc + v * 8 * LPR) = kr[v];
+          *reinterpret_cast<uint4*>(vc + v * 8 * LPR) = vr[v];
         }
       }
       float2 kf[4 * NV];
@@ -171,9 +182,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
 #pragma unroll
         for (int e = 0; e < 4 * NV; ++e) acc = __ffma2_rn(q[g][e], kf[e], acc);
         float x = acc.x + acc.y;
-        x += __shfl_xor_sync(0xffffffffu, x, 1);
-        x += __shfl_xor_sync(0xffffffffu, x, 2);
-        x += __shfl_xor_sync(0xffffffffu, x, 4);
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
         sc[g] = x;
       }
       if (valid) {
@@ -212,23 +222,25 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       mbar_wait(bar_full + 8 * (i % kDecStages), (i / kDecStages) & 1, p.err, ERR_WAIT_TMA);
   }
 
-  // ---- merge the four row groups of each warp with shuffles, then the four
-  // warps through shared memory (reusing the first stage's K tile)
+  // ---- merge the row groups of each warp with shuffles, then the four warps
+  // through shared memory (reusing the first stage's K tile)
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    float M = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], 8));
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
+    float M = m[g];
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     const float wgt = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - M);
     float lw = l[g] * wgt;
-    lw += __shfl_xor_sync(0xffffffffu, lw, 8);
-    lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
 #pragma unroll
     for (int e = 0; e < 4 * NV; ++e) {
       float x = o[g][e].x * wgt, y = o[g][e].y * wgt;
-      x += __shfl_xor_sync(0xffffffffu, x, 8);
-      x += __shfl_xor_sync(0xffffffffu, x, 16);
-      y += __shfl_xor_sync(0xffffffffu, y, 8);
-      y += __shfl_xor_sync(0xffffffffu, y, 16);
+#pragma unroll
+      for (int off = LPR; off < 32; off <<= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+        y += __shfl_xor_sync(0xffffffffu, y, off);
+      }
       o[g][e] = make_float2(x, y);
     }
     m[g] = M;
@@ -248,7 +260,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       for (int v = 0; v < NV; ++v)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int d = 64 * v + 8 * sub + 2 * e;
+          const int d = 8 * (sub + LPR * v) + 2 * e;
           sm_o[(warp * G + g) * D + d] = o[g][4 * v + e].x;
           sm_o[(warp * G + g) * D + d + 1] = o[g][4 * v + e].y;
         }
@@ -328,11 +340,25 @@ __global__ void decode_write_f32_kernel(const DecodeParams p) {
 }  // namespace
 
 int decode_chunks(int B, int Hkv, int W) {
-  // enough CTAs for ~16 per SM on 148 SMs, chunks of at least 2 pipeline stages
+  // Key chunks per (batch, KV head).  A CTA's time is about its rows plus a
+  // fixed cost (set-up, pipeline fill, partial write: ~2 stages of rows); the
+  // kernel's time is that times the number of waves of CTAs over 148 SMs with 4
+  // resident each.  Pick the count that minimises it, with chunks of at least
+  // 2 pipeline stages (at most 32 chunks).
   const int64_t pairs = static_cast<int64_t>(B) * Hkv;
-  int chunks = static_cast<int>((148LL * 16 + pairs - 1) / pairs);
-  chunks = imax(1, imin(chunks, cdiv(W, 2 * kDecRows)));
-  return chunks;
+  const int64_t slots = 148LL * 4;
+  const int cmax = imax(1, imin(32, cdiv(W, 2 * kDecRows)));
+  int best = 1;
+  double best_cost = 1e300;
+  for (int c = 1; c <= cmax; ++c) {
+    const int64_t waves = (pairs * c + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) * (static_cast<double>(W) / c + 2.0 * kDecRows);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = c;
+    }
+  }
+  return best;
 }
 
 int decode_chunk_len(int n_valid, int chunks) {
@@ -348,23 +374,31 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
 }
 
 namespace {
-template <int D, int G>
+template <int D, int G, int LPR, int ST>
 cudaError_t launch_dec(const DecodeParams& p, cudaStream_t stream) {
+  using PL = DecPlan<D, LPR, ST>;
   static int attr_dev_mask = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const int bit = 1 << (dev & 31);
   if (!(attr_dev_mask & bit)) {
-    const cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               DecPlan<D>::kSmemBytes);
+    const cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, LPR, ST>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_dev_mask |= bit;
   }
   dim3 grid(p.chunks, p.Hkv, p.B);
-  decode_kernel<D, G><<<grid, kDecThreads, DecPlan<D>::kSmemBytes, stream>>>(p);
+  decode_kernel<D, G, LPR, ST><<<grid, kDecThreads, PL::kSmemBytes, stream>>>(p);
   decode_combine_kernel<D><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
   count_launches(2);
   return cudaGetLastError();
+}
+template <int D, int G>
+cudaError_t launch_dec_pick(const DecodeParams& p, int lpr, cudaStream_t stream) {
+  if constexpr (D == 128) {
+    if (lpr == 16) return launch_dec<D, G, 16, 3>(p, stream);
+  }
+  return launch_dec<D, G, 8, 4>(p, stream);
 }
 }  // namespace
 
@@ -376,8 +410,16 @@ cudaError_t launch_decode_bf16(const DecodeParams& p_in, cudaStream_t stream) {
       !encode_rows_map(&p.tm_v, p.v_cache, p.D, p.Hkv, static_cast<int64_t>(p.B) * p.W, kDecRows))
     return cudaErrorInvalidValue;
   p.chunk_len = decode_chunk_len(p.n_valid, p.chunks);
+  // head_dim 128: 16 lanes per row, 3 stages (one chunk of q and O per lane and
+  // head, so four CTAs fit an SM by registers and shared memory); SWA_DEC_LPR=8
+  // selects 8 lanes per row and 4 stages (tuning).  head_dim 64: 8 lanes, 4 stages.
+  static int lpr = -1;
+  if (lpr < 0) {
+    const char* v = getenv("SWA_DEC_LPR");
+    lpr = (v && v[0] == '8') ? 8 : 16;
+  }
 #define SWA_DEC_CASE(DD, GG) \
-  if (p.D == DD && G == GG) return launch_dec<DD, GG>(p, stream);
+  if (p.D == DD && G == GG) return launch_dec_pick<DD, GG>(p, lpr, stream);
   SWA_DEC_CASE(128, 1) SWA_DEC_CASE(128, 2) SWA_DEC_CASE(128, 4) SWA_DEC_CASE(128, 8)
   SWA_DEC_CASE(64, 1) SWA_DEC_CASE(64, 2) SWA_DEC_CASE(64, 4) SWA_DEC_CASE(64, 8)
 #undef SWA_DEC_CASE
