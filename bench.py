@@ -263,11 +263,11 @@ def run_ours(args, rank, world, local_rank):
                               window_frames=ST["Wc"], page_tokens=ST["page"], max_frames=total_frames,
                               max_splits=12, device=dev)
 
-    def stream_frame(fr=None):
+    def stream_frame(fr=None, out=None):
         i = state["frame"]
         fq, fk, fv = frames[i % n_pool] if fr is None else fr
         cache.swa_stream_append_evict(0, i, fk, fv)
-        cache.swa_stream_attend(0, i, fq, sout)
+        cache.swa_stream_attend(0, i, fq, sout if out is None else out)
         state["frame"] = i + 1
 
     if use("stream"):
@@ -275,15 +275,15 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(ST["S"] + ST["Wc"]):
             stream_frame()
 
-    def prefill():
-        swa.swa_prefill(pq, pk, pv, pout, S=PF["F"], P=PF["P"], sliding_window_size=PF["sws"],
+    def prefill(q=pq, k=pk, v=pv, out=pout):
+        swa.swa_prefill(q, k, v, out, S=PF["F"], P=PF["P"], sliding_window_size=PF["sws"],
                         num_frame_per_block=PF["nfpb"], num_frame_for_scale=PF["S"])
 
-    def band():
-        swa.swa_band_prefill(bq, bk, bv, bout, window=BD["W"])
+    def band(q=bq, k=bk, v=bv, out=bout):
+        swa.swa_band_prefill(q, k, v, out, window=BD["W"])
 
-    def decode():
-        swa.swa_decode(dq, dkn, dvn, dkc, dvc, DC["pos"], dout, workspace=dws)
+    def decode(q=dq, k_new=dkn, v_new=dvn, out=dout):
+        swa.swa_decode(q, k_new, v_new, dkc, dvc, DC["pos"], out, workspace=dws)
 
     all_parts = [("prefill", prefill),
                  ("stream", lambda: [stream_frame() for _ in range(ST["frames_per_step"])]),
@@ -413,56 +413,95 @@ def run_ours(args, rank, world, local_rank):
 
 def run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn, dout,
             frames, sout, prefill, band, decode, stream_frame, world, dist, flops):
-    """Same step, timed with every input copied from pinned host memory and
-    every output copied back inside the timed region."""
-    fps = ST["frames_per_step"]
-    names = {n for n, _ in parts}
-    d_in = [t for t in (pq, pk, pv, bq, bk, bv, dq, dkn, dvn) if t is not None]
-    h_in = [t.cpu().pin_memory() for t in d_in]
-    use_stream = "stream" in names
-    h_frames = [tuple(t.cpu().pin_memory() for t in frames[j]) for j in range(fps)] if use_stream else []
-    d_frames = [tuple(torch.empty_like(t) for t in frames[j]) for j in range(fps)] if use_stream else []
-    d_out = [t for t in (pout, bout, dout) if t is not None]
-    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
-    h_sout = [torch.empty(sout.shape, dtype=sout.dtype, pin_memory=True) for _ in range(fps)] if use_stream else []
-    h2d = sum(t.numel() * t.element_size() for t in h_in) + sum(
-        t.numel() * t.element_size() for fr in h_frames for t in fr)
-    d2h = sum(t.numel() * t.element_size() for t in h_out) + sum(t.numel() * t.element_size() for t in h_sout)
-    outs = dict(zip([n for n, t in (("prefill", pout), ("band", bout), ("decode", dout)) if t is not None],
-                    zip(d_out, h_out)))
+    """The same step through the public API with every input copied from pinned
+    host memory and every output copied back, inside the timed region.
 
-    def e2e_step():
-        for h, d in zip(h_in, d_in):
-            d.copy_(h, non_blocking=True)
-        for name, fn in parts:
-            if name == "stream":
-                for j in range(fps):
-                    for h, d in zip(h_frames[j], d_frames[j]):
-                        d.copy_(h, non_blocking=True)
-                    stream_frame(d_frames[j])
-                    h_sout[j].copy_(sout, non_blocking=True)
-            else:
-                fn()
-                d, h = outs[name]
-                h.copy_(d, non_blocking=True)
+    Steps are pipelined the way a serving loop would run them: inputs and
+    outputs are double-buffered on the device, host-to-device copies run on one
+    stream, the attention calls on the compute stream and the read-backs on a
+    third, ordered by events, so step s+1's inputs arrive and step s-1's results
+    leave while step s computes.  The timed region runs from the first input
+    copy to the last read-back."""
+    fps = ST["frames_per_step"]
+    names = [n for n, _ in parts]
+    fns = {"prefill": prefill, "band": band, "decode": decode}
+    stage_io = {}
+    if "prefill" in names:
+        stage_io["prefill"] = ([pq, pk, pv], pout)
+    if "band" in names:
+        stage_io["band"] = ([bq, bk, bv], bout)
+    if "decode" in names:
+        stage_io["decode"] = ([dq, dkn, dvn], dout)
+    use_stream = "stream" in names
+    h_in = {n: [t.cpu().pin_memory() for t in ins] for n, (ins, _) in stage_io.items()}
+    h_out = {n: torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for n, (_, o) in stage_io.items()}
+    h_frames = [tuple(t.cpu().pin_memory() for t in frames[j]) for j in range(fps)] if use_stream else []
+    h_sout = [torch.empty(sout.shape, dtype=sout.dtype, pin_memory=True) for _ in range(fps)] if use_stream else []
+    d_in = [{n: [torch.empty_like(t) for t in ins] for n, (ins, _) in stage_io.items()} for _ in range(2)]
+    d_out = [{n: torch.empty_like(o) for n, (_, o) in stage_io.items()} for _ in range(2)]
+    d_frames = [[tuple(torch.empty_like(t) for t in frames[j]) for j in range(fps)] if use_stream else []
+                for _ in range(2)]
+    d_sout = [[torch.empty_like(sout) for _ in range(fps)] if use_stream else [] for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for ts in h_in.values() for t in ts) + sum(
+        t.numel() * t.element_size() for fr in h_frames for t in fr)
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values()) + sum(
+        t.numel() * t.element_size() for t in h_sout)
+
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(s):
+        k = s % 2
+        with torch.cuda.stream(s_in):
+            if s >= 2:
+                s_in.wait_event(ev_comp[k])  # step s-2 no longer reads input set k
+            for n, hs in h_in.items():
+                for h, d in zip(hs, d_in[k][n]):
+                    d.copy_(h, non_blocking=True)
+            for j in range(len(h_frames)):
+                for h, d in zip(h_frames[j], d_frames[k][j]):
+                    d.copy_(h, non_blocking=True)
+            ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if s >= 2:
+            stream.wait_event(ev_out[k])  # step s-2's results in output set k were read back
+        with torch.cuda.stream(stream):
+            for name, _ in parts:
+                if name == "stream":
+                    for j in range(fps):
+                        stream_frame(d_frames[k][j], d_sout[k][j])
+                else:
+                    fns[name](*d_in[k][name], d_out[k][name])
+            ev_comp[k].record(stream)
+        s_out.wait_event(ev_comp[k])
+        with torch.cuda.stream(s_out):
+            for n, h in h_out.items():
+                h.copy_(d_out[k][n], non_blocking=True)
+            for j in range(len(h_sout)):
+                h_sout[j].copy_(d_sout[k][j], non_blocking=True)
+            ev_out[k].record(s_out)
 
     steps = max(3, args.steps // 4)
-    e2e_step()
+    for s in range(2):
+        e2e_step(s)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    b.record(stream)
+    a.record(s_in)
+    for s in range(2, 2 + steps):
+        e2e_step(s)
+    b.record(s_out)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     ms = max_over_ranks(ms, world, dev)
     return {"value": weak_scaling_value(world, flops, steps, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": ms / steps}
+            "ms_per_step": ms / steps, "pipelined": "double-buffered inputs/outputs, copy-in / compute / "
+                                                    "copy-out streams"}
 
 
 # ---------------------------------------------------------------- oracle arm
