@@ -285,16 +285,27 @@ def run_ours(args, rank, world, local_rank):
     def decode(q=dq, k_new=dkn, v_new=dvn, out=dout):
         swa.swa_decode(q, k_new, v_new, dkc, dvc, DC["pos"], out, workspace=dws)
 
-    all_parts = [("prefill", prefill),
-                 ("stream", lambda: [stream_frame() for _ in range(ST["frames_per_step"])]),
-                 ("band", band), ("decode", decode)]
+    def stream_part(frame_evs=None):
+        # frame_evs: events around each frame (append + attend + combine) for
+        # per-frame latency percentiles
+        for j in range(ST["frames_per_step"]):
+            if frame_evs is not None:
+                frame_evs[j].record(stream)
+            stream_frame()
+        if frame_evs is not None:
+            frame_evs[ST["frames_per_step"]].record(stream)
+
+    all_parts = [("prefill", prefill), ("stream", stream_part), ("band", band), ("decode", decode)]
     parts = [(n, fn) for n, fn in all_parts if use(n)]
 
-    def step(evs=None):
-        for j, (_, fn) in enumerate(parts):
+    def step(evs=None, frame_evs=None):
+        for j, (name, fn) in enumerate(parts):
             if evs is not None:
                 evs[j].record(stream)
-            fn()
+            if name == "stream":
+                fn(frame_evs)
+            else:
+                fn()
         if evs is not None:
             evs[len(parts)].record(stream)
 
@@ -314,11 +325,13 @@ def run_ours(args, rank, world, local_rank):
     part_ms = {name: 0.0 for name, _ in parts}
     launches0 = swa.swa_launch_count()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(args.steps)]
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(ST["frames_per_step"] + 1)]
+           for _ in range(args.steps)] if use("stream") else [None] * args.steps
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for s in range(args.steps):
-        step(ev[s])
+        step(ev[s], fev[s])
     end.record(stream)
     torch.cuda.synchronize()
     launches = swa.swa_launch_count() - launches0
@@ -350,6 +363,10 @@ def run_ours(args, rank, world, local_rank):
         parts_out["stream_ms_per_frame"] = per["stream"] / ST["frames_per_step"]
         parts_out["stream_tflops"] = stage_flops["stream"] / (per["stream"] * 1e-3) / 1e12
         parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
+        lat = sorted(fev[s][j].elapsed_time(fev[s][j + 1]) for s in range(args.steps)
+                     for j in range(ST["frames_per_step"]))
+        parts_out["stream_frame_ms_p50"] = lat[len(lat) // 2]
+        parts_out["stream_frame_ms_p99"] = lat[min(len(lat) - 1, (99 * len(lat)) // 100)]
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
         parts_out["band_ms"] = per["band"]
