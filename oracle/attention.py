@@ -271,6 +271,31 @@ class StreamCache:
             out[:, h] = softmax_attention(q[:, h], kc[:, h], vc[:, h])
         return out
 
+    def attend_transient(self, layer: int, q, k, v) -> np.ndarray:
+        """Non-keyframe attend: the frame's queries [P, H, D] against everything
+        the layer's cache holds plus the frame's own keys/values [P, H, D], with
+        the cache left exactly as it was.
+
+        Follows the "Non-keyframe path" of the streaming branch in the pages'
+        block forward listing (lingbot-map AggregatorStream guide): the frame is
+        appended with eviction deferred, attended to, and the append is rolled
+        back.  So no frame is evicted (the oldest window frame is still visible),
+        no special token moves, and the frame counter does not advance."""
+        st = self.layers[layer]
+        k = np.asarray(k, dtype=np.float64)
+        v = np.asarray(v, dtype=np.float64)
+        q = np.asarray(q, dtype=np.float64)
+        if st.frames or st.specials_k:
+            kc, vc = self.gather(layer)
+            kc = np.concatenate([kc, k], axis=0)
+            vc = np.concatenate([vc, v], axis=0)
+        else:
+            kc, vc = k, v
+        out = np.zeros((q.shape[0], self.H, vc.shape[-1]))
+        for h in range(self.H):
+            out[:, h] = softmax_attention(q[:, h], kc[:, h], vc[:, h])
+        return out
+
     # --- exported bookkeeping ---------------------------------------------------
     def n_special_tokens(self, layer: int) -> int:
         return len(self.layers[layer].specials_k) * self.num_special

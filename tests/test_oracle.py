@@ -382,3 +382,71 @@ def test_frame_receptive_field_with_scale_frames():
             fi = i // P
             reachable = fi >= jf and (jf < S or fi - jf <= L * (Wf - 1))
             assert (not np.array_equal(out[i], base[i])) == reachable, (i, jf)
+
+
+# ---------------------------------------------------------------- non-keyframe attend
+def _frame(P, H, D, seed):
+    g = np.random.default_rng(seed)
+    return tuple(g.standard_normal((P, H, D)) for _ in range(3))
+
+
+def _state(cache, layer=0):
+    st = cache.layers[layer]
+    return (list(st.cached), sorted(st.frames), st.n_frames, st.n_evicted, st.last_evicted,
+            len(st.specials_k), cache.slot_frames(layer).tolist(), cache.page_table(layer).tolist())
+
+
+@pytest.mark.parametrize("special", [False, True])
+def test_transient_attend_equals_append_then_attend_before_any_eviction(special):
+    """While no eviction is due (fewer than S + W_c frames cached), appending a
+    frame and attending is exactly attending to the cache plus the frame."""
+    import copy
+    S, W, P, H, D = 2, 3, 7, 2, 4
+    cache = orc.StreamCache(H, D, P, S, W, page_tokens=4, cross_frame_special=special, num_special=2,
+                            max_frames=20)
+    for i in range(S + W):
+        q, k, v = _frame(P, H, D, 100 + i)
+        twin = copy.deepcopy(cache)
+        twin.append_evict(0, i, k, v)
+        assert twin.layers[0].last_evicted == -1
+        np.testing.assert_allclose(cache.attend_transient(0, q, k, v), twin.attend(0, q), atol=1e-12, rtol=0)
+        cache.append_evict(0, i, k, v)
+
+
+@pytest.mark.parametrize("special", [False, True])
+def test_transient_attend_leaves_cache_unchanged(special):
+    S, W, P, H, D = 1, 2, 6, 2, 4
+    cache = orc.StreamCache(H, D, P, S, W, page_tokens=4, cross_frame_special=special, num_special=2,
+                            max_frames=30)
+    for i in range(9):
+        q, k, v = _frame(P, H, D, 200 + i)
+        before = _state(cache)
+        cache.attend_transient(0, q, k, v)
+        assert _state(cache) == before
+        cache.append_evict(0, i, k, v)
+
+
+def test_transient_attend_sees_the_frame_a_keyframe_would_evict():
+    """Q = 0 gives uniform weights; V = one-hot of the key's frame id makes each
+    output column the fraction of keys from that frame.  A non-keyframe after
+    frame i sees scale frames, the window [i - W_c + 1, i] (eviction deferred:
+    frame i - W_c + 1 stays) and itself; the keyframe i + 1 sees one frame
+    fewer (i + 1 - W_c is evicted)."""
+    S, W, P, H = 1, 3, 5, 1
+    F = 8
+    D = F + 1  # one-hot over frame ids 0..F (id F: the non-keyframe)
+    cache = orc.StreamCache(H, D, P, S, W, page_tokens=4, max_frames=20)
+    z = np.zeros((P, H, D))
+    for i in range(F):
+        v = np.zeros((P, H, D))
+        v[:, :, i] = 1.0
+        cache.append_evict(0, i, z, v)
+    i = F - 1
+    vt = np.zeros((P, H, D))
+    vt[:, :, F] = 1.0
+    got = cache.attend_transient(0, z, z, vt)[0, 0]
+    frames = list(range(S)) + list(range(i - W + 1, i + 1)) + [F]
+    want = np.zeros(D)
+    want[frames] = 1.0 / len(frames)
+    np.testing.assert_allclose(got, want, atol=1e-15, rtol=0)
+    assert 1.0 / len(frames) == pytest.approx(1.0 / (S + W + 1))
