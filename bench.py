@@ -367,6 +367,25 @@ def run_ours(args, rank, world, local_rank):
                      for j in range(ST["frames_per_step"]))
         parts_out["stream_frame_ms_p50"] = lat[len(lat) // 2]
         parts_out["stream_frame_ms_p99"] = lat[min(len(lat) - 1, (99 * len(lat)) // 100)]
+        # the non-keyframe path at the same steady state (timed apart from the
+        # step): the frame attends to the cache plus itself, nothing persists,
+        # so its keys are 8 scale + 64 window + 1 frames
+        tq, tk, tv = frames[0]
+        nk_out = torch.empty_like(sout)
+        for _ in range(3):
+            cache.swa_stream_attend_transient(0, tq, tk, tv, nk_out)
+        n_nk = 8
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_nk):
+            cache.swa_stream_attend_transient(0, tq, tk, tv, nk_out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        nk_ms = e0.elapsed_time(e1) / n_nk
+        nk_flops = flops_stream_frame() * (ST["S"] + ST["Wc"] + 1) / (ST["S"] + ST["Wc"])
+        parts_out["stream_nonkey_ms_per_frame"] = nk_ms
+        parts_out["stream_nonkey_frames_per_s"] = 1e3 / nk_ms
+        parts_out["stream_nonkey_tflops"] = nk_flops / (nk_ms * 1e-3) / 1e12
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
         parts_out["band_ms"] = per["band"]

@@ -165,6 +165,22 @@ swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx,
 swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx,
                              const void* q_frame, void* out, void* stream);
 
+/* Non-keyframe attend ("Non-keyframe path" of the streaming attention block,
+ * lingbot-map AggregatorStream guide: append with eviction deferred, attend,
+ * roll the append back).  The queries q_frame [P, heads, head_dim] attend to
+ * everything the layer's cache holds after its last keyframe (retained full
+ * frames and specials, nothing evicted on this frame's account) plus this
+ * frame's own k_frame, v_frame [P, heads, head_dim]; out [P, heads, head_dim].
+ * Nothing persistent changes: the frame's K/V go to a scratch frame of pages
+ * that no page table lists, the frame counter does not advance, no frame or
+ * special token moves.  Valid on an empty layer (the frame attends to itself).
+ * Shares the split-KV partials and the scratch frame with the handle's other
+ * calls: calls on one handle must not overlap on the GPU.  Errors: SWA_ERR_ARG
+ * (null or misaligned pointer), SWA_ERR_CAPACITY (global_idx out of range). */
+swa_status swa_stream_attend_transient(swa_stream* h, int global_idx, const void* q_frame,
+                                       const void* k_frame, const void* v_frame, void* out,
+                                       void* stream);
+
 /* Layout of one layer's metadata block, in int32 units. */
 typedef struct swa_meta_layout {
     int n_ints;          /* size of the block                                  */

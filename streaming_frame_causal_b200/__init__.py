@@ -64,6 +64,7 @@ _sigs = {
     "swa_stream_reset": (_i, [_vp, _vp]),
     "swa_stream_append_evict": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "swa_stream_attend": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "swa_stream_attend_transient": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
     "swa_stream_get_meta": (_i, [_vp, _i, _vp, _sz, _vp]),
     "swa_stream_k_storage": (_vp, [_vp, _i]),
@@ -281,6 +282,14 @@ class SwaStream:
     def swa_stream_attend(self, global_idx: int, frame_idx: int, q_frame, out, stream=None):
         _check(_lib.swa_stream_attend(self.handle, global_idx, frame_idx, _ptr(q_frame), _ptr(out),
                                       _stream(stream)), "swa_stream_attend")
+        return out
+
+    def swa_stream_attend_transient(self, global_idx: int, q_frame, k_frame, v_frame, out, stream=None):
+        """Non-keyframe attend: q_frame against the cache plus this frame's own
+        K/V, with nothing persisted (see include/swa.h)."""
+        _check(_lib.swa_stream_attend_transient(self.handle, global_idx, _ptr(q_frame), _ptr(k_frame),
+                                                _ptr(v_frame), _ptr(out), _stream(stream)),
+               "swa_stream_attend_transient")
         return out
 
     def swa_stream_get_meta(self, global_idx: int, stream=None) -> dict:

@@ -385,6 +385,8 @@ extern "C" swa_status swa_decode(const void* q, const void* k_new, const void* v
 struct swa_stream {
   swa_stream_cfg cfg;
   int n_slots, ppf, special_pages, max_pages, max_segs;
+  int scratch_page;  // first page of the non-keyframe scratch frame (after the special region)
+  int t_off;         // offset (ints) of the non-keyframe header + key runs in a layer's metadata
   int64_t total_rows;
   int row_bytes;
   int meta_ints;
@@ -403,7 +405,7 @@ namespace {
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct StreamGeom {
-  int n_slots, ppf, special_pages, max_pages, max_segs, meta_ints, row_bytes;
+  int n_slots, ppf, special_pages, max_pages, max_segs, meta_ints, row_bytes, scratch_page, t_off;
   int64_t total_rows;
   size_t meta_stride, store_bytes, part_bytes, total;
 };
@@ -424,12 +426,16 @@ bool stream_geom(const swa_stream_cfg* c, StreamGeom* g) {
   const int64_t sp_tokens = c->cross_frame_special ? static_cast<int64_t>(max_evicted) * c->num_special : 0;
   g->special_pages = static_cast<int>(cdiv(static_cast<int>(sp_tokens), c->page_tokens));
   const int64_t pages = static_cast<int64_t>(g->n_slots) * g->ppf + g->special_pages;
-  if (pages * c->page_tokens > 0x7fffffffLL) return false;
+  // one more frame of pages after the special region: the non-keyframe scratch frame
+  if ((pages + g->ppf) * c->page_tokens > 0x7fffffffLL) return false;
   g->max_pages = static_cast<int>(pages);
+  g->scratch_page = static_cast<int>(pages);
   g->max_segs = g->n_slots + 1;
-  g->total_rows = pages * c->page_tokens;
+  g->total_rows = (pages + g->ppf) * c->page_tokens;
   g->meta_ints = 8 + g->n_slots + g->max_pages + 2 * g->max_segs;
-  g->meta_stride = round256(static_cast<size_t>(g->meta_ints) * 4);
+  // non-keyframe area after the published layout: header + key runs (one more run)
+  g->t_off = g->meta_ints;
+  g->meta_stride = round256(static_cast<size_t>(g->meta_ints + 8 + 2 * (g->max_segs + 1)) * 4);
   g->store_bytes = round256(static_cast<size_t>(g->total_rows) * g->row_bytes);
   const size_t rows_h = static_cast<size_t>(c->P) * c->heads;
   g->part_bytes = round256(static_cast<size_t>(c->max_splits) * rows_h * c->head_dim * 4) +
@@ -475,6 +481,8 @@ extern "C" swa_status swa_stream_create(swa_stream** out, const swa_stream_cfg* 
   h->max_pages = g.max_pages;
   h->max_segs = g.max_segs;
   h->total_rows = g.total_rows;
+  h->scratch_page = g.scratch_page;
+  h->t_off = g.t_off;
   h->row_bytes = g.row_bytes;
   h->meta_ints = g.meta_ints;
   h->meta_stride = g.meta_stride;
@@ -589,28 +597,25 @@ int choose_splits(int T, int items_per_split, int max_splits, int sms) {
 
 }  // namespace
 
-extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
-                                        void* out, void* stream) {
-  swa_status s = stream_check_layer(h, global_idx);
-  if (s != SWA_OK) return s;
-  if (!q_frame || !out || !aligned16(q_frame) || !aligned16(out)) return SWA_ERR_ARG;
-  if (h->n_frames[global_idx] == 0 || frame_idx != h->n_frames[global_idx] - 1) return SWA_ERR_ORDER;
+namespace {
+// The attend of a frame's queries against key runs listed in device metadata:
+// hdr (n_segs at hdr[5]), run rows and lengths, at most max_segs runs, which
+// cover n_frames_keys full frames plus n_special special tokens.
+swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame, void* out, cudaStream_t st,
+                              const int* hdr, const int* seg_row, const int* seg_len, int max_segs,
+                              int n_frames_keys, int n_special) {
   int* err = err_ptr();
   if (!err) return SWA_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const swa_stream_cfg& c = h->cfg;
-  int* meta = layer_meta(h, global_idx);
-  const int off_seg_row = 8 + h->n_slots + h->max_pages;
-  const int off_seg_len = off_seg_row + h->max_segs;
   if (c.dtype == SWA_F32) {
     SimtParams p{};
     p.q = static_cast<const float*>(q_frame);
     p.k = reinterpret_cast<const float*>(layer_k(h, global_idx));
     p.v = reinterpret_cast<const float*>(layer_v(h, global_idx));
     p.out = static_cast<float*>(out);
-    p.seg_row = meta + off_seg_row;
-    p.seg_len = meta + off_seg_len;
-    p.meta_hdr = meta;
+    p.seg_row = seg_row;
+    p.seg_len = seg_len;
+    p.meta_hdr = hdr;
     p.err = err;
     p.mode = SIMT_STREAM;
     p.B = 1;
@@ -619,15 +624,11 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
     p.Hq = c.heads;
     p.Hkv = c.heads;
     p.D = c.head_dim;
-    p.max_segs = h->max_segs;
+    p.max_segs = max_segs;
     p.scale = 1.f / std::sqrt(static_cast<float>(c.head_dim));
     return cuda_status(launch_attn_simt(p, st));
   }
-  const int i = frame_idx;
-  const int n_ret = stream_retained(i, c.scale_frames, c.window_frames);
-  const int n_special =
-      c.cross_frame_special ? stream_n_evicted(i, c.scale_frames, c.window_frames) * c.num_special : 0;
-  const int T = n_ret * cdiv(c.P, kTileRows) + cdiv(n_special, kTileRows);
+  const int T = n_frames_keys * cdiv(c.P, kTileRows) + cdiv(n_special, kTileRows);
   const int n_pairs = qpairs_per_frame(c.P);
   const int items = c.heads * n_pairs;
   const int splits = choose_splits(T, items, c.max_splits, num_sms());
@@ -639,9 +640,9 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
   p.out = out;
   p.part_o = h->part_o;
   p.part_ml = h->part_ml;
-  p.seg_row = meta + off_seg_row;
-  p.seg_len = meta + off_seg_len;
-  p.meta_hdr = meta;
+  p.seg_row = seg_row;
+  p.seg_len = seg_len;
+  p.meta_hdr = hdr;
   p.err = err;
   p.mode = TC_STREAM;
   p.B = 1;
@@ -651,12 +652,71 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
   p.P = c.P;
   p.n_pairs = n_pairs;
   p.splits = splits;
-  p.max_segs = h->max_segs;
+  p.max_segs = max_segs;
   p.scale_log2 = scale_log2(c.head_dim);
   cudaError_t e = launch_attn_tc(p, c.head_dim, static_cast<int64_t>(items) * splits, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
   if (splits > 1) e = launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, c.head_dim, splits, st);
   return cuda_status(e);
+}
+}  // namespace
+
+extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
+                                        void* out, void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  if (!q_frame || !out || !aligned16(q_frame) || !aligned16(out)) return SWA_ERR_ARG;
+  if (h->n_frames[global_idx] == 0 || frame_idx != h->n_frames[global_idx] - 1) return SWA_ERR_ORDER;
+  const swa_stream_cfg& c = h->cfg;
+  int* meta = layer_meta(h, global_idx);
+  const int off_seg_row = 8 + h->n_slots + h->max_pages;
+  const int off_seg_len = off_seg_row + h->max_segs;
+  const int i = frame_idx;
+  const int n_ret = stream_retained(i, c.scale_frames, c.window_frames);
+  const int n_special =
+      c.cross_frame_special ? stream_n_evicted(i, c.scale_frames, c.window_frames) * c.num_special : 0;
+  return stream_attend_impl(h, global_idx, q_frame, out, static_cast<cudaStream_t>(stream), meta,
+                            meta + off_seg_row, meta + off_seg_len, h->max_segs, n_ret, n_special);
+}
+
+extern "C" swa_status swa_stream_attend_transient(swa_stream* h, int global_idx, const void* q_frame,
+                                                  const void* k_frame, const void* v_frame, void* out,
+                                                  void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  if (!q_frame || !k_frame || !v_frame || !out || !aligned16(q_frame) || !aligned16(k_frame) ||
+      !aligned16(v_frame) || !aligned16(out))
+    return SWA_ERR_ARG;
+  int* err = err_ptr();
+  if (!err) return SWA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const swa_stream_cfg& c = h->cfg;
+  int* meta = layer_meta(h, global_idx);
+  TransientParams tp{};
+  tp.k_src = static_cast<const uint8_t*>(k_frame);
+  tp.v_src = static_cast<const uint8_t*>(v_frame);
+  tp.k_store = layer_k(h, global_idx);
+  tp.v_store = layer_v(h, global_idx);
+  tp.meta = meta;
+  tp.err = err;
+  tp.P = c.P;
+  tp.row_bytes = c.heads * c.head_dim * (c.dtype == SWA_F32 ? 4 : 2);
+  tp.page_tokens = c.page_tokens;
+  tp.scratch_page = h->scratch_page;
+  tp.off_seg_row = 8 + h->n_slots + h->max_pages;
+  tp.off_seg_len = tp.off_seg_row + h->max_segs;
+  tp.max_segs = h->max_segs;
+  tp.t_off = h->t_off;
+  if (launch_transient_prepare(tp, st) != cudaSuccess) return SWA_ERR_CUDA;
+  // keys: the frames and specials the cache holds after its last keyframe, plus this frame
+  const int nf = h->n_frames[global_idx];
+  const int n_ret = nf > 0 ? stream_retained(nf - 1, c.scale_frames, c.window_frames) : 0;
+  const int n_special = (nf > 0 && c.cross_frame_special)
+                            ? stream_n_evicted(nf - 1, c.scale_frames, c.window_frames) * c.num_special
+                            : 0;
+  int* th = meta + h->t_off;
+  return stream_attend_impl(h, global_idx, q_frame, out, st, th, th + 8, th + 8 + (h->max_segs + 1),
+                            h->max_segs + 1, n_ret + 1, n_special);
 }
 
 extern "C" swa_status swa_stream_meta_layout(const swa_stream* h, swa_meta_layout* out) {

@@ -115,6 +115,48 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
   }
 }
 
+// Non-keyframe attend ("Non-keyframe path" of the streaming block in the same
+// guide: append with eviction deferred, attend, roll back): the frame's K/V are
+// written to the scratch frame's pages, which no persistent page table lists,
+// and the layer's non-keyframe area receives the persistent key runs followed by
+// the scratch run.  Nothing persistent is written, so the roll-back is free.
+__global__ void __launch_bounds__(256) transient_prepare_kernel(const TransientParams p) {
+  const int chunks = p.row_bytes >> 4;
+  const int64_t per_tensor = static_cast<int64_t>(p.P) * chunks;
+  const int64_t row0 = static_cast<int64_t>(p.scratch_page) * p.page_tokens;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < 2 * per_tensor;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int tsel = static_cast<int>(idx / per_tensor);
+    const int64_t rem = idx - tsel * per_tensor;
+    const int row = static_cast<int>(rem / chunks);
+    const int ch = static_cast<int>(rem - static_cast<int64_t>(row) * chunks);
+    uint8_t* store = tsel ? p.v_store : p.k_store;
+    const uint8_t* src = tsel ? p.v_src : p.k_src;
+    reinterpret_cast<uint4*>(store + (row0 + row) * p.row_bytes)[ch] =
+        reinterpret_cast<const uint4*>(src + static_cast<int64_t>(row) * p.row_bytes)[ch];
+  }
+  if (blockIdx.x != 0) return;
+  const int* hdr = p.meta;
+  int* th = p.meta + p.t_off;
+  int* trow = th + 8;
+  int* tlen = trow + (p.max_segs + 1);
+  int n = hdr[5];
+  if (n < 0 || n > p.max_segs) {
+    if (threadIdx.x == 0) atomicOr(p.err, ERR_BAD_META);
+    n = 0;
+  }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    trow[e] = hdr[p.off_seg_row + e];
+    tlen[e] = hdr[p.off_seg_len + e];
+  }
+  if (threadIdx.x == 0) {
+    trow[n] = static_cast<int>(row0);
+    tlen[n] = p.P;
+    for (int e = 0; e < 8; ++e) th[e] = hdr[e];
+    th[5] = n + 1;
+  }
+}
+
 __global__ void debug_wait_kernel(int* err, long long timeout_ns) {
   // waits on a flag that nothing sets; gives up after timeout_ns and latches
   // the error -- the same bounded-wait contract every kernel follows
@@ -157,6 +199,16 @@ cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
   if (blocks < 1) blocks = 1;
   if (blocks > 4096) blocks = 4096;
   append_evict_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transient_prepare(const TransientParams& p, cudaStream_t stream) {
+  const int64_t work = 2LL * p.P * (p.row_bytes >> 4);
+  int64_t blocks = (work + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 4096) blocks = 4096;
+  transient_prepare_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -75,6 +75,22 @@ struct AppendParams {
 
 cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream);
 
+// Non-keyframe attend, preparation: the frame's K/V go to the scratch frame's
+// pages, and the layer's non-keyframe area gets the persistent key runs plus the
+// scratch run (the persistent metadata is only read).
+struct TransientParams {
+  const uint8_t* k_src;  // [P, H, D] of the non-keyframe
+  const uint8_t* v_src;
+  uint8_t* k_store;      // page storage [total_rows, H, D]
+  uint8_t* v_store;
+  int* meta;             // the layer's metadata block
+  int* err;              // device error flag
+  int P, row_bytes, page_tokens, scratch_page;
+  int off_seg_row, off_seg_len, max_segs, t_off;
+};
+
+cudaError_t launch_transient_prepare(const TransientParams& p, cudaStream_t stream);
+
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
   CUtensorMap tm_k;   // K cache as rows [B*W, Hkv, D], box = 32 rows x 1 head x D

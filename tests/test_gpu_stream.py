@@ -147,3 +147,91 @@ def test_1000_frame_stream_with_specials(swa):
     rows = np.unique(np.concatenate([np.arange(0, 1004, 53), [0, 4, 5, 1003]]))
     _stream(swa, F=1000, P=1004, H=16, D=64, S=8, Wc=64, special=True, dtype=torch.bfloat16,
             frames_to_check={72, 500, 999}, check_rows=rows)
+
+
+# ---------------------------------------------------------------- non-keyframe attend
+def _raw_meta(cache, layer=0):
+    m = cache.swa_stream_get_meta(layer)
+    return {k: (v.tolist() if hasattr(v, "tolist") else v) for k, v in m.items()}
+
+
+def _transient_stream(swa, F, P, H, D, S, Wc, special, dtype, at, check_rows=None, keyframes=None):
+    """Keyframes 0..F-1; before each keyframe listed in ``at`` (F: after the
+    last) a non-keyframe with its own seeded Q/K/V attends through the cache
+    without persisting.  Its output matches the oracle, the metadata is
+    bit-identical before and after it, and the keyframes listed in
+    ``keyframes`` (default: all) still match the oracle.  With ``check_rows``
+    the oracle is evaluated on those query rows only."""
+    dev = "cuda"
+    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
+                          cross_frame_special=special, num_special=5, max_frames=F, dtype=dtype)
+    oc = orc.StreamCache(heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, page_tokens=16,
+                         cross_frame_special=special, num_special=5, max_frames=F)
+    check = check_f32 if dtype == torch.float32 else check_bf16
+    rows = np.arange(P) if check_rows is None else np.asarray(check_rows)
+
+    def ref_rows(q, extra=None):
+        # oracle attention of the sampled query rows against the cache (+ extra K/V)
+        if oc.layers[0].frames or oc.layers[0].specials_k:
+            kc, vc = oc.gather(0)
+            if extra is not None:
+                kc, vc = np.concatenate([kc, extra[0]]), np.concatenate([vc, extra[1]])
+        else:
+            kc, vc = extra
+        qq = q[rows]
+        return np.stack([orc.softmax_attention(qq[:, h], kc[:, h], vc[:, h]) for h in range(H)], 1)
+
+    for i in range(F + 1):
+        if i in at:
+            tq, tk, tv = synth.stream_frame(10_000 + i, P=P, H=H, D=D, dtype=dtype, base_seed=7)
+            before = _raw_meta(cache) if i > 0 else None
+            out = torch.empty(tq.shape, dtype=dtype, device=dev)
+            cache.swa_stream_attend_transient(0, tq.to(dev), tk.to(dev), tv.to(dev), out)
+            torch.cuda.synchronize()
+            got = out.float().cpu().numpy()[rows]
+            if check_rows is None:
+                ref = oc.attend_transient(0, tq.float().numpy(), tk.float().numpy(), tv.float().numpy())
+            else:
+                ref = ref_rows(tq.float().numpy(), (tk.float().numpy(), tv.float().numpy()))
+            check(got, ref, f"non-keyframe before keyframe {i}")
+            if before is not None:
+                assert _raw_meta(cache) == before
+        if i == F:
+            break
+        q, k, v = synth.stream_frame(i, P=P, H=H, D=D, dtype=dtype)
+        cache.swa_stream_append_evict(0, i, k.to(dev), v.to(dev))
+        oc.append_evict(0, i, k.float().numpy(), v.float().numpy())
+        _compare_meta(cache.swa_stream_get_meta(0), oc, 0, i)
+        if keyframes is not None and i not in keyframes:
+            continue
+        out = torch.empty(q.shape, dtype=dtype, device=dev)
+        cache.swa_stream_attend(0, i, q.to(dev), out)
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()[rows]
+        ref = oc.attend(0, q.float().numpy()) if check_rows is None else ref_rows(q.float().numpy())
+        check(got, ref, f"keyframe {i}")
+    assert swa.swa_device_error_check() == 0
+
+
+@pytest.mark.parametrize("special", [False, True])
+def test_transient_attend_bf16(swa, special):
+    """2 scale + 3 window frames of 200 tokens (two query tiles), 2 x 64: the
+    non-keyframe on an empty cache, while the window fills, once it is full
+    (the frame a keyframe would evict is still visible), and late in the stream."""
+    _transient_stream(swa, F=10, P=200, H=2, D=64, S=2, Wc=3, special=special, dtype=torch.bfloat16,
+                      at={0, 1, 4, 5, 6, 9, 10})
+
+
+def test_transient_attend_head_dim_128_and_f32(swa):
+    _transient_stream(swa, F=7, P=130, H=2, D=128, S=1, Wc=2, special=True, dtype=torch.bfloat16,
+                      at={0, 3, 5, 7})
+    _transient_stream(swa, F=6, P=21, H=2, D=32, S=1, Wc=2, special=True, dtype=torch.float32,
+                      at={0, 2, 4, 6})
+
+
+def test_transient_attend_full_size(swa):
+    """8 scale + 64 window frames of 1004 tokens, 16 x 64: a non-keyframe after
+    80 keyframes (73 frames of keys), checked on sampled rows."""
+    rows = np.unique(np.concatenate([np.arange(0, 1004, 61), [127, 128, 1003]]))
+    _transient_stream(swa, F=80, P=1004, H=16, D=64, S=8, Wc=64, special=False, dtype=torch.bfloat16,
+                      at={79, 80}, check_rows=rows, keyframes={79})
