@@ -27,13 +27,15 @@ def _compare_meta(meta, oc, layer, i):
 
 
 def _stream(swa, F, P, H, D, S, Wc, special, dtype, frames_to_check, max_frames=None, layers=1,
-            check_rows=None):
+            check_rows=None, num_special=5):
     max_frames = max_frames or F
     dev = "cuda"
     cache = swa.SwaStream(num_layers=layers, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
-                          cross_frame_special=special, num_special=5, max_frames=max_frames, dtype=dtype)
+                          cross_frame_special=special, num_special=num_special, max_frames=max_frames,
+                          dtype=dtype)
     oc = orc.StreamCache(heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, page_tokens=16,
-                         cross_frame_special=special, num_special=5, max_frames=max_frames, num_layers=layers)
+                         cross_frame_special=special, num_special=num_special, max_frames=max_frames,
+                         num_layers=layers)
     for i in range(F):
         for layer in range(layers):
             q, k, v = synth.stream_frame(i, P=P, H=H, D=D, dtype=dtype, base_seed=layer)
@@ -235,3 +237,19 @@ def test_transient_attend_full_size(swa):
     rows = np.unique(np.concatenate([np.arange(0, 1004, 61), [127, 128, 1003]]))
     _transient_stream(swa, F=80, P=1004, H=16, D=64, S=8, Wc=64, special=False, dtype=torch.bfloat16,
                       at={79, 80}, check_rows=rows, keyframes={79})
+
+
+def test_camera_only_retention(swa):
+    """Evicted frames keep only their camera token (num_special = 1, the reading
+    taken for kv_cache_camera_only): bookkeeping bit-exact, attention matches."""
+    _stream(swa, F=12, P=300, H=2, D=64, S=2, Wc=3, special=True, dtype=torch.bfloat16,
+            frames_to_check=set(range(12)), num_special=1)
+
+
+def test_no_scale_frames(swa):
+    """No protected scale frames (scale_frames = 0, the reading taken for
+    kv_cache_include_scale_frames=False): a pure window of frames."""
+    _stream(swa, F=10, P=300, H=2, D=64, S=0, Wc=3, special=False, dtype=torch.bfloat16,
+            frames_to_check=set(range(10)))
+    _stream(swa, F=10, P=300, H=2, D=64, S=0, Wc=3, special=True, dtype=torch.bfloat16,
+            frames_to_check={3, 6, 9})

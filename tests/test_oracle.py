@@ -227,17 +227,23 @@ def _tiny_stream(S, W, F, P, H, D, special, ns, seed):
     return q, k, v, np.concatenate(outs, axis=0)
 
 
-def test_stream_equals_prefill_tiny_config():
+@pytest.mark.parametrize("S", [2, 0])
+def test_stream_equals_prefill_tiny_config(S):
     """The 8-frame, 21-token, 2x32 check case: frame-by-frame streaming through
-    the rolling cache reproduces the full-sequence masked attention."""
-    S, W, F, P, H, D = 2, 3, 8, 21, 2, 32
+    the rolling cache reproduces the full-sequence masked attention.  S = 0 is
+    the cache without protected scale frames (the reading taken for
+    kv_cache_include_scale_frames=False): a pure frame window."""
+    W, F, P, H, D = 3, 8, 21, 2, 32
     q, k, v, streamed = _tiny_stream(S, W, F, P, H, D, False, 5, 100)
     full = orc.prefill(q[None], k[None], v[None], P=P, scale_frames=S, sliding_window_size=W)[0]
     np.testing.assert_allclose(streamed, full, atol=1e-12, rtol=0)
 
 
-def test_special_retention_equals_extended_mask():
-    S, W, F, P, H, D, ns = 1, 2, 7, 7, 2, 4, 2
+@pytest.mark.parametrize("ns", [2, 1])
+def test_special_retention_equals_extended_mask(ns):
+    """Evicted frames keep their first ns tokens.  ns = 1 keeps the camera token
+    only (the reading taken for kv_cache_camera_only)."""
+    S, W, F, P, H, D = 1, 2, 7, 7, 2, 4
     q, k, v, streamed = _tiny_stream(S, W, F, P, H, D, True, ns, 200)
     N = F * P
     for i in range(F):
