@@ -18,8 +18,12 @@ Sources (page title, section):
          append_frame -> evict_frames -> compute_attention, q/k/v in [tpf, H, D].
   [SWA]  sliding-window attention explainer (Mistral 7B): band i-W+1..i,
          rolling buffer slot i mod W, grouped-query attention, L*W reach.
+  [PRE]  "Method forward" (block forward listing): the compiled attn_pre step
+         "norm1 + qkv linear + reshape + q_norm + k_norm + RoPE + format", and
+         the I/O page's 3-D RoPE format: a complex-valued table
+         [.., S_global*P, head_dim/2] (WanRotaryPosEmbed).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
   * causality is frame-granular: a query frame sees all of its own frame
     ([AGG] snippet ends the window at the end of the current frame);
   * the first ``S = num_frame_for_scale`` frames are always visible to later
@@ -29,7 +33,11 @@ Readings where the pages are silent (each listed in the design doc):
     in [AGG] "Mask Generation");
   * the special tokens of a frame are its first ``num_special`` tokens
     (camera, then registers), and evicted frames keep them in cache order of
-    eviction.
+    eviction;
+  * attn_pre: norm1 is a LayerNorm over C with weight and bias, the qkv linear
+    has a bias, q_norm / k_norm are LayerNorms over head_dim with weight and
+    bias, and RoPE multiplies the (2i, 2i+1) pairs of q and k by the caller's
+    complex table (cos, sin) per token and pair.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (closed forms, library special cases, brute force on tiny inputs, the pages'
@@ -392,3 +400,49 @@ def decode(q, k_new, v_new, k_cache, v_cache, pos: int, W: int):
             out[b, h] = softmax_attention(q[b, h][None, :], kc[b, :n_valid, g],
                                           vc[b, :n_valid, g])[0]
     return out, kc, vc
+
+
+# ----------------------------------------------------------------------------
+# attn_pre prologue  ([PRE]: norm1 + qkv linear + reshape + q_norm + k_norm + RoPE)
+# ----------------------------------------------------------------------------
+def layer_norm(x, weight, bias, eps: float):
+    """LayerNorm over the last axis: (x - mean) / sqrt(var + eps) * weight + bias
+    (biased variance), in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(weight, np.float64) + np.asarray(bias, np.float64)
+
+
+def rope_complex(x, rot):
+    """Rotate the (2i, 2i+1) pairs of x [..., P, H, D] by the complex numbers
+    rot [P, D/2, 2] = (cos, sin) of each token and pair: the complex-valued
+    position format of the I/O page's 3-D RoPE (x viewed as D/2 complex
+    numbers, multiplied elementwise)."""
+    x = np.asarray(x, dtype=np.float64)
+    rot = np.asarray(rot, dtype=np.float64)
+    re, im = x[..., 0::2], x[..., 1::2]
+    c = rot[:, None, :, 0]  # broadcast over heads
+    s = rot[:, None, :, 1]
+    out = np.empty_like(x)
+    out[..., 0::2] = re * c - im * s
+    out[..., 1::2] = re * s + im * c
+    return out
+
+
+def attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads: int, eps: float = 1e-6):
+    """One frame's attention prologue ([PRE]): x [P, C] -> q, k, v [P, H, D].
+
+    norm1 (LayerNorm over C) -> qkv linear (x_n @ w_qkv.T + b_qkv, w_qkv
+    [3C, C]) -> reshape to [P, 3, H, D] -> q_norm, k_norm (LayerNorm over D) ->
+    RoPE on q and k (complex pairs, table rot [P, D/2, 2]); v is passed on."""
+    x = np.asarray(x, dtype=np.float64)
+    P, C = x.shape
+    D = C // heads
+    xn = layer_norm(x, ln_w, ln_b, eps)
+    qkv = xn @ np.asarray(w_qkv, np.float64).T + np.asarray(b_qkv, np.float64)
+    qkv = qkv.reshape(P, 3, heads, D)
+    q = layer_norm(qkv[:, 0], qn_w, qn_b, eps)
+    k = layer_norm(qkv[:, 1], kn_w, kn_b, eps)
+    v = qkv[:, 2]
+    return rope_complex(q, rot), rope_complex(k, rot), v.copy()

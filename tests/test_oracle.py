@@ -456,3 +456,100 @@ def test_transient_attend_sees_the_frame_a_keyframe_would_evict():
     want[frames] = 1.0 / len(frames)
     np.testing.assert_allclose(got, want, atol=1e-15, rtol=0)
     assert 1.0 / len(frames) == pytest.approx(1.0 / (S + W + 1))
+
+
+# ---------------------------------------------------------------- attn_pre prologue
+def _prologue_inputs(P=6, H=2, D=8, seed=5):
+    g = np.random.default_rng(seed)
+    C = H * D
+    x = g.standard_normal((P, C)) * 3 + 1
+    w = dict(ln_w=1 + 0.1 * g.standard_normal(C), ln_b=0.1 * g.standard_normal(C),
+             w_qkv=g.standard_normal((3 * C, C)) / np.sqrt(C), b_qkv=0.1 * g.standard_normal(3 * C),
+             qn_w=1 + 0.1 * g.standard_normal(D), qn_b=0.1 * g.standard_normal(D),
+             kn_w=1 + 0.1 * g.standard_normal(D), kn_b=0.1 * g.standard_normal(D))
+    ang = g.uniform(-np.pi, np.pi, (P, D // 2))
+    rot = np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+    return x, w, rot, ang
+
+
+def test_layer_norm_matches_torch_and_row_statistics():
+    x, w, _, _ = _prologue_inputs()
+    eps = 1e-6
+    got = orc.layer_norm(x, w["ln_w"], w["ln_b"], eps)
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (x.shape[1],), torch.from_numpy(w["ln_w"]),
+                                         torch.from_numpy(w["ln_b"]), eps).numpy()
+    np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
+    plain = orc.layer_norm(x, np.ones(x.shape[1]), np.zeros(x.shape[1]), eps)
+    var = x.var(axis=1)
+    np.testing.assert_allclose(plain.mean(axis=1), 0, atol=1e-13)
+    np.testing.assert_allclose((plain ** 2).mean(axis=1), var / (var + eps), rtol=1e-12)
+
+
+def test_rope_complex_matches_torch_complex_product():
+    g = np.random.default_rng(8)
+    P, H, D = 5, 3, 8
+    x = g.standard_normal((P, H, D))
+    ang = g.uniform(-3, 3, (P, D // 2))
+    rot = np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+    xt = torch.view_as_complex(torch.from_numpy(x).reshape(P, H, D // 2, 2).contiguous())
+    ref = torch.view_as_real(xt * torch.polar(torch.ones(P, 1, D // 2, dtype=torch.float64),
+                                              torch.from_numpy(ang)[:, None, :])).reshape(P, H, D).numpy()
+    np.testing.assert_allclose(orc.rope_complex(x, rot), ref, atol=1e-12, rtol=0)
+
+
+def test_rope_identity_norms_and_relative_positions():
+    g = np.random.default_rng(9)
+    P, H, D = 7, 2, 8
+    x = g.standard_normal((P, H, D))
+    ident = np.stack([np.ones((P, D // 2)), np.zeros((P, D // 2))], axis=-1)
+    np.testing.assert_array_equal(orc.rope_complex(x, ident), x)
+    # a frequency per pair, position p -> angle p * omega: rotated q_m . k_n depends on n - m only
+    omega = 10.0 ** (-np.arange(D // 2) / (D // 2))
+    def table(pos):
+        a = np.outer(pos, omega)
+        return np.stack([np.cos(a), np.sin(a)], axis=-1)
+    q, k = g.standard_normal((1, H, D)), g.standard_normal((1, H, D))
+    def dot(m, n):
+        return np.sum(orc.rope_complex(q, table([m])) * orc.rope_complex(k, table([n])))
+    for m, n, t in [(0, 3, 5), (2, -4, 11), (7, 7, -3)]:
+        assert dot(m, n) == pytest.approx(dot(m + t, n + t), abs=1e-12)
+    r = orc.rope_complex(x, table(np.arange(P)))
+    np.testing.assert_allclose(np.linalg.norm(r, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+
+
+def test_attn_pre_matches_torch_restatement():
+    x, w, rot, ang = _prologue_inputs()
+    P, C = x.shape
+    H, D = 2, C // 2
+    eps = 1e-6
+    q, k, v = orc.attn_pre(x, w["ln_w"], w["ln_b"], w["w_qkv"], w["b_qkv"], w["qn_w"], w["qn_b"],
+                           w["kn_w"], w["kn_b"], rot, heads=H, eps=eps)
+    T = {n: torch.from_numpy(a) for n, a in w.items()}
+    F = torch.nn.functional
+    xn = F.layer_norm(torch.from_numpy(x), (C,), T["ln_w"], T["ln_b"], eps)
+    qkv = F.linear(xn, T["w_qkv"], T["b_qkv"]).reshape(P, 3, H, D)
+    tq = F.layer_norm(qkv[:, 0], (D,), T["qn_w"], T["qn_b"], eps)
+    tk = F.layer_norm(qkv[:, 1], (D,), T["kn_w"], T["kn_b"], eps)
+    rotc = torch.polar(torch.ones(P, 1, D // 2, dtype=torch.float64), torch.from_numpy(ang)[:, None, :])
+    def rope(t):
+        return torch.view_as_real(torch.view_as_complex(t.reshape(P, H, D // 2, 2).contiguous()) * rotc
+                                  ).reshape(P, H, D)
+    np.testing.assert_allclose(q, rope(tq).numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(k, rope(tk).numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(v, qkv[:, 2].numpy(), atol=1e-12, rtol=0)
+
+
+def test_attn_pre_head_norms_closed_form():
+    """Unit norm weights, zero norm biases: each rotated q/k head vector has squared
+    norm D * s2 / (s2 + eps), s2 the variance of that head of the linear output."""
+    x, w, rot, _ = _prologue_inputs(seed=11)
+    P, C = x.shape
+    H, D = 2, C // 2
+    eps = 1e-6
+    one, zero = np.ones(D), np.zeros(D)
+    q, k, _ = orc.attn_pre(x, w["ln_w"], w["ln_b"], w["w_qkv"], w["b_qkv"], one, zero, one, zero, rot,
+                           heads=H, eps=eps)
+    lin = (orc.layer_norm(x, w["ln_w"], w["ln_b"], eps) @ w["w_qkv"].T + w["b_qkv"]).reshape(P, 3, H, D)
+    for t, out in ((0, q), (1, k)):
+        s2 = lin[:, t].var(axis=-1)
+        np.testing.assert_allclose((out ** 2).sum(axis=-1), D * s2 / (s2 + eps), rtol=1e-12)
