@@ -386,6 +386,27 @@ def run_ours(args, rank, world, local_rank):
         parts_out["stream_nonkey_ms_per_frame"] = nk_ms
         parts_out["stream_nonkey_frames_per_s"] = 1e3 / nk_ms
         parts_out["stream_nonkey_tflops"] = nk_flops / (nk_ms * 1e-3) / 1e12
+        # the attention prologue of a streaming frame (norm1, qkv linear on the
+        # tensor cores, q/k norms, RoPE), timed apart from the step
+        Cm = ST["H"] * ST["D"]
+        pin = {k: t.to(dev) for k, t in synth.prologue_inputs(seed=9, P=ST["P"], C=Cm, heads=ST["H"]).items()}
+        pre_args = [pin[n] for n in ("ln_w", "ln_b", "w_qkv", "b_qkv", "qn_w", "qn_b", "kn_w", "kn_b", "rot")]
+        pre_out = [torch.empty(ST["P"], ST["H"], ST["D"], dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        pre_ws = torch.empty_like(pin["x"])
+        def pre():
+            swa.swa_attn_pre(pin["x"], *pre_args, heads=ST["H"], q_out=pre_out[0], k_out=pre_out[1],
+                             v_out=pre_out[2], xn_ws=pre_ws)
+        for _ in range(3):
+            pre()
+        n_pre = 20
+        e0.record(stream)
+        for _ in range(n_pre):
+            pre()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pre_ms = e0.elapsed_time(e1) / n_pre
+        parts_out["prologue_us"] = pre_ms * 1e3
+        parts_out["prologue_qkv_tflops"] = 2.0 * ST["P"] * Cm * 3 * Cm / (pre_ms * 1e-3) / 1e12
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
         parts_out["band_ms"] = per["band"]

@@ -181,6 +181,38 @@ swa_status swa_stream_attend_transient(swa_stream* h, int global_idx, const void
                                        const void* k_frame, const void* v_frame, void* out,
                                        void* stream);
 
+/* Attention prologue of one frame ("Method forward", block forward listing: the
+ * compiled attn_pre step "norm1 + qkv linear + reshape + q_norm + k_norm + RoPE +
+ * format"; RoPE in the I/O page's complex-valued format).  Readings for the steps
+ * the listing names without defining: norm1 = LayerNorm over C with weight ln_w
+ * and bias ln_b, qkv = norm1(x) w_qkv^T + b_qkv, q_norm / k_norm = LayerNorm over
+ * head_dim of each head with weights qn_w / kn_w and biases qn_b / kn_b, all with
+ * epsilon eps (biased variance); RoPE multiplies the (2i, 2i+1) element pairs of
+ * every q and k head by the complex number rot[p][i] = (cos, sin) of its token p.
+ *   x      [P, C] bf16 (C = heads * head_dim, C a multiple of 256, C <= 2048,
+ *          head_dim 64 or 128)          w_qkv [3C, C] bf16 (rows q | k | v)
+ *   ln_w, ln_b [C], b_qkv [3C], qn_w, qn_b, kn_w, kn_b [head_dim], rot [P, head_dim/2, 2]: f32
+ *   xn_ws  [P, C] bf16 workspace (norm1 output)
+ *   q_out, k_out, v_out [P, heads, head_dim] bf16.
+ * All device pointers, 16-byte aligned, caller-owned.  Errors: SWA_ERR_ARG (null or
+ * misaligned pointer, negative size, eps <= 0), SWA_ERR_UNSUPPORTED (shape). */
+swa_status swa_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
+                        const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
+                        const float* kn_b, const float* rot, int P, int C, int heads, float eps,
+                        void* xn_ws, void* q_out, void* k_out, void* v_out, void* stream);
+
+/* Streaming append with the prologue fused in: the eviction and metadata of
+ * swa_stream_append_evict for frame ``frame_idx``, then swa_attn_pre on the frame's
+ * tokens x [P, C] with K and V written straight into the frame's slot of the
+ * layer's page storage (no separate K/V frame), Q to q_out [P, heads, head_dim] for
+ * swa_stream_attend.  bf16 caches only; C = heads * head_dim of the cache.  Errors
+ * as swa_stream_append_evict and swa_attn_pre. */
+swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
+                                       const float* ln_w, const float* ln_b, const void* w_qkv,
+                                       const float* b_qkv, const float* qn_w, const float* qn_b,
+                                       const float* kn_w, const float* kn_b, const float* rot, float eps,
+                                       void* xn_ws, void* q_out, void* stream);
+
 /* Layout of one layer's metadata block, in int32 units. */
 typedef struct swa_meta_layout {
     int n_ints;          /* size of the block                                  */

@@ -65,6 +65,8 @@ _sigs = {
     "swa_stream_append_evict": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "swa_stream_attend": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "swa_stream_attend_transient": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
+    "swa_attn_pre": (_i, [_vp] * 10 + [_i, _i, _i, C.c_float] + [_vp] * 5),
+    "swa_stream_append_evict_pre": (_i, [_vp, _i, _i] + [_vp] * 10 + [C.c_float] + [_vp] * 3),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
     "swa_stream_get_meta": (_i, [_vp, _i, _vp, _sz, _vp]),
     "swa_stream_k_storage": (_vp, [_vp, _i]),
@@ -159,6 +161,23 @@ def swa_prefill(q, k, v, out, S: int, P: int, sliding_window_size: int, num_fram
                             sliding_window_size, num_frame_per_block, num_frame_for_scale,
                             _dtype_code(q), _stream(stream)), "swa_prefill")
     return out
+
+
+def swa_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads: int, eps: float = 1e-6,
+                 q_out=None, k_out=None, v_out=None, xn_ws=None, stream=None):
+    """Attention prologue of one frame: x [P, C] bf16 -> q, k, v [P, heads, C/heads]
+    bf16 (norm1, qkv linear, q/k norms, RoPE by the complex table rot [P, D/2, 2];
+    the steps and layouts are those of swa_attn_pre in include/swa.h)."""
+    P, Cdim = x.shape
+    D = Cdim // heads
+    q_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if q_out is None else q_out
+    k_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if k_out is None else k_out
+    v_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if v_out is None else v_out
+    xn_ws = torch.empty_like(x) if xn_ws is None else xn_ws
+    _check(_lib.swa_attn_pre(_ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv), _ptr(qn_w), _ptr(qn_b),
+                             _ptr(kn_w), _ptr(kn_b), _ptr(rot), P, Cdim, heads, float(eps), _ptr(xn_ws),
+                             _ptr(q_out), _ptr(k_out), _ptr(v_out), _stream(stream)), "swa_attn_pre")
+    return q_out, k_out, v_out
 
 
 def swa_band_prefill(q, k, v, out, window: int, stream=None) -> torch.Tensor:
@@ -283,6 +302,18 @@ class SwaStream:
         _check(_lib.swa_stream_attend(self.handle, global_idx, frame_idx, _ptr(q_frame), _ptr(out),
                                       _stream(stream)), "swa_stream_attend")
         return out
+
+    def swa_stream_append_evict_pre(self, global_idx: int, frame_idx: int, x, ln_w, ln_b, w_qkv, b_qkv, qn_w,
+                                    qn_b, kn_w, kn_b, rot, q_out, eps: float = 1e-6, xn_ws=None, stream=None):
+        """Append frame ``frame_idx`` from its tokens x [P, C]: eviction and
+        metadata, then the attention prologue with K/V written into the frame's
+        slot and Q to q_out [P, heads, head_dim] (see include/swa.h)."""
+        xn_ws = torch.empty_like(x) if xn_ws is None else xn_ws
+        _check(_lib.swa_stream_append_evict_pre(self.handle, global_idx, frame_idx, _ptr(x), _ptr(ln_w), _ptr(ln_b),
+                                                _ptr(w_qkv), _ptr(b_qkv), _ptr(qn_w), _ptr(qn_b), _ptr(kn_w),
+                                                _ptr(kn_b), _ptr(rot), float(eps), _ptr(xn_ws), _ptr(q_out),
+                                                _stream(stream)), "swa_stream_append_evict_pre")
+        return q_out
 
     def swa_stream_attend_transient(self, global_idx: int, q_frame, k_frame, v_frame, out, stream=None):
         """Non-keyframe attend: q_frame against the cache plus this frame's own

@@ -108,6 +108,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+bool swa::encode_2d_sw128(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool swa::encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -538,15 +550,9 @@ extern "C" swa_status swa_stream_reset(swa_stream* h, void* stream) {
   return SWA_OK;
 }
 
-extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx, const void* k_frame,
-                                              const void* v_frame, void* stream) {
-  swa_status s = stream_check_layer(h, global_idx);
-  if (s != SWA_OK) return s;
-  if (!k_frame || !v_frame || !aligned16(k_frame) || !aligned16(v_frame)) return SWA_ERR_ARG;
-  if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
-  if (frame_idx >= h->cfg.max_frames) return SWA_ERR_CAPACITY;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+namespace {
+AppendParams append_params(swa_stream* h, int global_idx, int frame_idx, const void* k_frame,
+                           const void* v_frame, int* err) {
   AppendParams p{};
   p.k_src = static_cast<const uint8_t*>(k_frame);
   p.v_src = static_cast<const uint8_t*>(v_frame);
@@ -570,10 +576,112 @@ extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int
   p.off_seg_len = p.off_seg_row + h->max_segs;
   p.max_pages = h->max_pages;
   p.max_segs = h->max_segs;
+  p.copy = 1;
+  return p;
+}
+}  // namespace
+
+extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx, const void* k_frame,
+                                              const void* v_frame, void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  if (!k_frame || !v_frame || !aligned16(k_frame) || !aligned16(v_frame)) return SWA_ERR_ARG;
+  if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
+  if (frame_idx >= h->cfg.max_frames) return SWA_ERR_CAPACITY;
+  int* err = err_ptr();
+  if (!err) return SWA_ERR_CUDA;
+  const AppendParams p = append_params(h, global_idx, frame_idx, k_frame, v_frame, err);
   const cudaError_t e = launch_append_evict(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return SWA_ERR_CUDA;
   h->n_frames[global_idx] = frame_idx + 1;
   return SWA_OK;
+}
+
+// ================================================================ attn_pre prologue
+namespace {
+bool pre_shape_ok(int P, int C, int heads) {
+  if (P < 0 || heads < 1 || C < 1 || C % heads) return false;
+  const int D = C / heads;
+  return (D == 64 || D == 128) && C % 256 == 0 && C <= 2048;
+}
+
+swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
+                        const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
+                        const float* kn_b, const float* rot, int P, int C, int heads, float eps, void* xn_ws,
+                        void* q_out, uint8_t* k_dst, uint8_t* v_dst, cudaStream_t st) {
+  int* err = err_ptr();
+  if (!err) return SWA_ERR_CUDA;
+  if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
+  PreParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_2d_sw128(&p.tm_a, xn_ws, C, P, 128) || !encode_2d_sw128(&p.tm_b, w_qkv, C, 3LL * C, 256))
+    return SWA_ERR_CUDA;
+  p.b_qkv = b_qkv;
+  p.qn_w = qn_w;
+  p.qn_b = qn_b;
+  p.kn_w = kn_w;
+  p.kn_b = kn_b;
+  p.rot = rot;
+  p.q_out = q_out;
+  p.k_dst = k_dst;
+  p.v_dst = v_dst;
+  p.kv_row_bytes = static_cast<int64_t>(C) * 2;
+  p.err = err;
+  p.P = P;
+  p.C = C;
+  p.H = heads;
+  p.D = C / heads;
+  p.eps = eps;
+  return cuda_status(launch_qkv_pre(p, st));
+}
+}  // namespace
+
+extern "C" swa_status swa_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
+                                   const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
+                                   const float* kn_b, const float* rot, int P, int C, int heads, float eps,
+                                   void* xn_ws, void* q_out, void* k_out, void* v_out, void* stream) {
+  if (!pre_shape_ok(P, C, heads)) return (P < 0 || heads < 1 || C < 1) ? SWA_ERR_ARG : SWA_ERR_UNSUPPORTED;
+  if (!(eps > 0.f)) return SWA_ERR_ARG;
+  if (P == 0) return SWA_OK;
+  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, xn_ws, q_out, k_out, v_out};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return SWA_ERR_ARG;
+  return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, P, C, heads, eps, xn_ws, q_out,
+                      static_cast<uint8_t*>(k_out), static_cast<uint8_t*>(v_out), static_cast<cudaStream_t>(stream));
+}
+
+extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
+                                                  const float* ln_w, const float* ln_b, const void* w_qkv,
+                                                  const float* b_qkv, const float* qn_w, const float* qn_b,
+                                                  const float* kn_w, const float* kn_b, const float* rot, float eps,
+                                                  void* xn_ws, void* q_out, void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  const swa_stream_cfg& c = h->cfg;
+  if (c.dtype != SWA_BF16) return SWA_ERR_UNSUPPORTED;
+  const int C = c.heads * c.head_dim;
+  if (!pre_shape_ok(c.P, C, c.heads)) return SWA_ERR_UNSUPPORTED;
+  if (!(eps > 0.f)) return SWA_ERR_ARG;
+  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, xn_ws, q_out};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return SWA_ERR_ARG;
+  if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
+  if (frame_idx >= c.max_frames) return SWA_ERR_CAPACITY;
+  int* err = err_ptr();
+  if (!err) return SWA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // eviction (the evicted frame's specials leave its slot first) and metadata,
+  // then the prologue writes the frame's K/V into that slot
+  AppendParams ap = append_params(h, global_idx, frame_idx, nullptr, nullptr, err);
+  ap.copy = 0;
+  if (launch_append_evict(ap, st) != cudaSuccess) return SWA_ERR_CUDA;
+  h->n_frames[global_idx] = frame_idx + 1;
+  const int64_t slot_row0 = static_cast<int64_t>(stream_slot(frame_idx, c.scale_frames, c.window_frames)) *
+                            h->ppf * c.page_tokens;
+  uint8_t* kd = layer_k(h, global_idx) + slot_row0 * h->row_bytes;
+  uint8_t* vd = layer_v(h, global_idx) + slot_row0 * h->row_bytes;
+  return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, c.P, C, c.heads, eps, xn_ws,
+                      q_out, kd, vd, st);
 }
 
 namespace {

@@ -71,6 +71,8 @@ struct AppendParams {
   int row_bytes;         // H * D * element size (multiple of 16)
   int off_slot_frame, off_page_table, off_seg_row, off_seg_len;
   int max_pages, max_segs;
+  int copy;              // 0: move specials and rewrite metadata only (the frame's K/V
+                         // are written into its slot by the attn_pre prologue)
 };
 
 cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream);
@@ -113,6 +115,31 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
 int decode_chunk_len(int n_valid, int chunks);
 // bf16 [rows, H, D] as a 3-D tensor map with a box of box_rows rows of one head (no swizzle)
 bool encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows);
+// bf16 matrix [rows, inner] (inner contiguous) as a 2-D map; box = 64 columns x
+// box_rows rows, 128-byte swizzle
+bool encode_2d_sw128(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int box_rows);
+
+// ---------------------------------------------------------------- attn_pre prologue
+struct PreParams {
+  CUtensorMap tm_a;     // norm1 output [P, C] bf16, box 64 x 128
+  CUtensorMap tm_b;     // w_qkv [3C, C] bf16, box 64 x 256
+  const float* b_qkv;   // [3C]
+  const float* qn_w;    // [D] q_norm weight / bias
+  const float* qn_b;
+  const float* kn_w;    // [D] k_norm weight / bias
+  const float* kn_b;
+  const float* rot;     // [P, D/2, 2]: (cos, sin) per token and pair
+  void* q_out;          // [P, H, D] bf16
+  uint8_t* k_dst;       // K rows: [P, H, D] at row stride k_row_bytes (a buffer or cache slot rows)
+  uint8_t* v_dst;
+  int64_t kv_row_bytes; // H * D * 2
+  int* err;
+  int P, C, H, D;
+  float eps;
+};
+cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
+                           cudaStream_t stream);
+cudaError_t launch_qkv_pre(const PreParams& p, cudaStream_t stream);
 int decode_chunks(int B, int Hkv, int W);
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);

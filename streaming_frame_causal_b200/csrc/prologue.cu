@@ -1,0 +1,282 @@
+// prologue.cu -- the attention prologue of a streaming frame ("Method forward",
+// block forward listing: the compiled attn_pre step "norm1 + qkv linear +
+// reshape + q_norm + k_norm + RoPE + format"), written as two kernels:
+//
+//   ln_rows_kernel   norm1: LayerNorm over C of each token, bf16 out
+//   qkv_pre_kernel   qkv = norm1(x) @ w_qkv^T + b_qkv on the tensor cores
+//                    (tcgen05, TMA-fed 4-stage ring, accumulator in TMEM), and
+//                    in the epilogue, per 128-token x 256-feature tile: the bias,
+//                    per-head LayerNorm of the q and k sections, RoPE on q and k
+//                    (the (2i, 2i+1) pairs times the caller's complex table: the
+//                    I/O page's complex-valued 3-D RoPE format), bf16 stores.
+//                    K and V can go straight into a frame slot of the paged
+//                    cache, so the streaming append needs no second copy.
+//
+// Readings where the listing names a step but not its form: LayerNorms with
+// weight and bias and a caller-given epsilon, a qkv bias, RoPE as a complex
+// product with a per-token table [P, D/2] of (cos, sin).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tile_sched.h"
+
+namespace swa {
+namespace {
+
+// ---------------------------------------------------------------- norm1
+// One warp per token row; each lane owns the 16-byte chunks lane, lane + 32, ...
+__global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                      const float* __restrict__ w, const float* __restrict__ b,
+                                                      __nv_bfloat16* __restrict__ out, int P, int C, float eps) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= P) return;
+  constexpr int kMaxChunks = 8;  // C <= 2048
+  const int nch = C / 256;       // 8-element chunks per lane
+  const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * C;
+  float v[kMaxChunks * 8];
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (c >= nch) break;
+    const uint4 u = *reinterpret_cast<const uint4*>(xr + (c * 32 + lane) * 8);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[c * 8 + 2 * e] = __uint_as_float(w4[e] << 16);
+      v[c * 8 + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+      s += v[c * 8 + 2 * e] + v[c * 8 + 2 * e + 1];
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float mean = s / C;
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (c >= nch) break;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float d = v[c * 8 + e] - mean;
+      q += d * d;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+  const float rs = rsqrtf(q / C + eps);
+  __nv_bfloat16* orow = out + static_cast<int64_t>(row) * C;
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (c >= nch) break;
+    const int col = (c * 32 + lane) * 8;
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a0 = (v[c * 8 + 2 * e] - mean) * rs * __ldg(w + col + 2 * e) + __ldg(b + col + 2 * e);
+      const float a1 = (v[c * 8 + 2 * e + 1] - mean) * rs * __ldg(w + col + 2 * e + 1) + __ldg(b + col + 2 * e + 1);
+      o[e] = pack_bf16x2(a0, a1);
+    }
+    *reinterpret_cast<uint4*>(orow + col) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ---------------------------------------------------------------- qkv GEMM
+constexpr int kPreThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int kPreM = 128;        // tokens per tile
+constexpr int kPreN = 256;        // output features per tile
+constexpr int kPreStages = 4;
+constexpr int kPreABytes = kPreM * 64 * 2;  // 16 KB: 128 rows x 64 columns
+constexpr int kPreBBytes = kPreN * 64 * 2;  // 32 KB
+constexpr int kPreStageBytes = kPreABytes + kPreBBytes;
+constexpr int kPreOffBar = kPreStages * kPreStageBytes;
+constexpr int kPreSmem = kPreOffBar + (2 * kPreStages + 1) * 8 + 16 + 1024;
+
+template <int D>
+__global__ void __launch_bounds__(kPreThreads, 1) qkv_pre_kernel(const __grid_constant__ PreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw_base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kPreM;
+  const int n0 = blockIdx.y * kPreN;
+  const int KC = p.C / 64;  // 64-column chunks of the reduction
+  const uint32_t bar0 = base + kPreOffBar;
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kPreStages + s); };
+  const uint32_t acc_full = bar0 + 8u * (2 * kPreStages);
+  const uint32_t tmem_slot = acc_full + 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPreStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kPreN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + (tmem_slot - base));
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_a);
+      tma_prefetch_desc(&p.tm_b);
+      int issued = 0;
+      for (int kc = 0; kc < KC; ++kc) {
+        const int s = kc % kPreStages;
+        if (kc >= kPreStages && !mbar_wait(empty(s), ((kc / kPreStages) - 1) & 1, p.err, ERR_WAIT_TMA)) break;
+        const uint32_t dst = base + s * kPreStageBytes;
+        mbar_arrive_expect_tx(full(s), kPreStageBytes);
+        tma_load_2d(dst, &p.tm_a, full(s), kc * 64, m0);
+        tma_load_2d(dst + kPreABytes, &p.tm_b, full(s), kc * 64, n0);
+        ++issued;
+      }
+      for (int kc = issued - kPreStages; kc < issued; ++kc) {
+        if (kc < 0) continue;
+        mbar_wait(full(kc % kPreStages), (kc / kPreStages) & 1, p.err, ERR_WAIT_TMA);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPreM, kPreN, 0);
+      const uint64_t da0 = sdesc_sw128(base, 16, 1024);
+      const uint64_t db0 = sdesc_sw128(base + kPreABytes, 16, 1024);
+      bool ok = true;
+      for (int kc = 0; kc < KC && ok; ++kc) {
+        const int s = kc % kPreStages;
+        if (!mbar_wait(full(s), (kc / kPreStages) & 1, p.err, ERR_WAIT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t step = static_cast<uint64_t>(s * (kPreStageBytes >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem, da0 + step + 2 * kk, db0 + step + 2 * kk, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(empty(s));
+      }
+      mma_commit(acc_full);
+      mbar_wait(acc_full, 0, p.err, ERR_WAIT_MMA);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;
+    const int row = m0 + r;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.err, ERR_WAIT_EPI));
+    if (ok) {
+      tc_fence_after();
+      const int sec = n0 / p.C;            // 0: q, 1: k, 2: v
+      const int h0 = (n0 - sec * p.C) / D;  // first head of this tile
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const float* nw = sec == 0 ? p.qn_w : p.kn_w;
+      const float* nb = sec == 0 ? p.qn_b : p.kn_b;
+#pragma unroll 1
+      for (int hh = 0; hh < kPreN / D; ++hh) {
+        __syncwarp();  // tcgen05.ld is warp-collective: all lanes converged
+        uint32_t a[D];
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(tmem + lane_off + hh * D + c0, a + c0);
+        tmem_wait_ld();
+        if (row < p.P) {
+        const int fcol = n0 + hh * D;  // first output feature of this head
+        float v[D];
+#pragma unroll
+        for (int j = 0; j < D; ++j) v[j] = __uint_as_float(a[j]) + __ldg(p.b_qkv + fcol + j);
+        if (sec < 2) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < D; ++j) s += v[j];
+          const float mean = s / D;
+          float q = 0.f;
+#pragma unroll
+          for (int j = 0; j < D; ++j) q += (v[j] - mean) * (v[j] - mean);
+          const float rs = rsqrtf(q / D + p.eps);
+#pragma unroll
+          for (int j = 0; j < D; ++j) v[j] = (v[j] - mean) * rs * __ldg(nw + j) + __ldg(nb + j);
+          const float2* rt = reinterpret_cast<const float2*>(p.rot) + static_cast<int64_t>(row) * (D / 2);
+#pragma unroll
+          for (int i = 0; i < D / 2; ++i) {
+            const float2 cs = __ldg(rt + i);
+            const float x0 = v[2 * i], x1 = v[2 * i + 1];
+            v[2 * i] = x0 * cs.x - x1 * cs.y;
+            v[2 * i + 1] = x0 * cs.y + x1 * cs.x;
+          }
+        }
+        const int h = h0 + hh;
+        uint8_t* dst;
+        if (sec == 0)
+          dst = reinterpret_cast<uint8_t*>(p.q_out) + (static_cast<int64_t>(row) * p.H + h) * D * 2;
+        else
+          dst = (sec == 1 ? p.k_dst : p.v_dst) + static_cast<int64_t>(row) * p.kv_row_bytes + h * D * 2;
+#pragma unroll
+        for (int j = 0; j < D; j += 8) {
+          uint4 u;
+          u.x = pack_bf16x2(v[j], v[j + 1]);
+          u.y = pack_bf16x2(v[j + 2], v[j + 3]);
+          u.z = pack_bf16x2(v[j + 4], v[j + 5]);
+          u.w = pack_bf16x2(v[j + 6], v[j + 7]);
+          *reinterpret_cast<uint4*>(dst + j * 2) = u;
+        }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kPreN);
+  }
+}
+
+template <int D>
+cudaError_t launch_pre_d(const PreParams& p, cudaStream_t stream) {
+  static int attr_dev_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const int bit = 1 << (dev & 31);
+  if (!(attr_dev_mask & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(qkv_pre_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmem);
+    if (e != cudaSuccess) return e;
+    attr_dev_mask |= bit;
+  }
+  dim3 grid(cdiv(p.P, kPreM), 3 * p.C / kPreN);
+  qkv_pre_kernel<D><<<grid, kPreThreads, kPreSmem, stream>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
+                           cudaStream_t stream) {
+  if (P <= 0) return cudaSuccess;
+  ln_rows_kernel<<<cdiv(P, 8), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), w, b,
+                                                  static_cast<__nv_bfloat16*>(out), P, C, eps);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qkv_pre(const PreParams& p, cudaStream_t stream) {
+  if (p.P <= 0) return cudaSuccess;
+  if (p.D == 64) return launch_pre_d<64>(p, stream);
+  if (p.D == 128) return launch_pre_d<128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace swa

@@ -146,3 +146,26 @@ def growing_scores_qkv(seed: int = 7, P: int = 1000, H: int = 2, D: int = 64, st
     k = tile_beta / (D ** 0.5) * torch.ones(1, P, H, D) + noise * torch.randn(1, P, H, D, generator=g)
     v = torch.randn(1, P, H, D, generator=g)
     return q.to(dtype), k.to(dtype), v.to(dtype)
+
+
+def prologue_inputs(seed: int = 3, P: int = P_FRAME, C: int = C_MODEL, heads: int = HEADS,
+                    x_dtype=torch.bfloat16):
+    """Inputs of one frame's attention prologue: tokens x [P, C] ~ N(0, 1) (bf16),
+    norm weights ~ 1 + N(0, 0.1^2) and biases ~ N(0, 0.1^2) (f32), w_qkv [3C, C] ~
+    N(0, 1/C) (bf16), b_qkv ~ N(0, 0.02^2) (f32), and a rotation table rot
+    [P, D/2, 2] = (cos, sin) of angle p * 100^(-i/(D/2)) for token p and pair i
+    (f32).  Returns a dict of CPU tensors."""
+    g = _gen(seed)
+    D = C // heads
+    r = lambda *s: torch.randn(*s, generator=g, dtype=torch.float32)
+    ang = torch.arange(P, dtype=torch.float64)[:, None] * (100.0 ** (-torch.arange(D // 2, dtype=torch.float64)
+                                                                     / (D // 2)))[None, :]
+    rot = torch.stack([torch.cos(ang), torch.sin(ang)], dim=-1).to(torch.float32)
+    return {
+        "x": r(P, C).to(x_dtype),
+        "ln_w": 1 + 0.1 * r(C), "ln_b": 0.1 * r(C),
+        "w_qkv": (r(3 * C, C) / C ** 0.5).to(torch.bfloat16), "b_qkv": 0.02 * r(3 * C),
+        "qn_w": 1 + 0.1 * r(D), "qn_b": 0.1 * r(D),
+        "kn_w": 1 + 0.1 * r(D), "kn_b": 0.1 * r(D),
+        "rot": rot.contiguous(),
+    }
