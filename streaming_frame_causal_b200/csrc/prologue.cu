@@ -28,6 +28,16 @@
 namespace swa {
 namespace {
 
+// 2-D tiled TMA load into shared memory (x = innermost coordinate, in elements;
+// x times the element size must be a multiple of 16 bytes)
+SWA_DEV void tma_load_2d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(mbar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- norm1
 // One warp per token row; each lane owns the 16-byte chunks lane, lane + 32, ...
 __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __restrict__ x,

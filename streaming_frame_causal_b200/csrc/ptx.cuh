@@ -90,16 +90,6 @@ SWA_DEV void tma_prefetch_desc(const void* tmap) {
 // 4-D tiled bulk tensor load global -> shared, completion counted on ``mbar``.
 // c0 is the innermost (contiguous) coordinate and must be a multiple of 8 for
 // 16-bit elements (16-byte rule); the callers only pass 0 or 64.
-// 2-D tiled TMA load into shared memory (x = innermost coordinate, in elements;
-// x times the element size must be a multiple of 16 bytes)
-SWA_DEV void tma_load_2d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(mbar)
-      : "memory");
-}
-
 SWA_DEV void tma_load_4d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, int c1, int c2,
                          int c3) {
   asm volatile(
