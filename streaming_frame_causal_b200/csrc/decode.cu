@@ -51,6 +51,45 @@ SWA_DEV void tma_load_3d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, 
       : "memory");
 }
 
+// Sum each of the G per-lane partial scores x[g] over the LPR lanes of a row
+// group, leaving every lane with all G sums.  Butterfly with halving: at the
+// level with xor offset LPR/2^k the lanes whose offset bit is set keep the upper
+// half of their remaining heads and send the lower half (and the other way
+// round), so after log2(G) levels each lane holds one head's partial sum over
+// 2^log2(G) lanes; the remaining offsets finish that sum, and G shuffles from
+// the lanes owning each head broadcast the results.  log2(G) + G - 1 + log2(LPR/G)
+// shuffles per group instead of G log2(LPR).
+template <int G, int LPR>
+SWA_DEV void reduce_heads(float (&x)[G], int lane) {
+  static_assert(G <= LPR, "at most one head per lane of a row group");
+  float v[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) v[g] = x[g];
+#pragma unroll
+  for (int n = G, off = LPR / 2; n > 1; n >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+    const int half = n / 2;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? v[i] : v[half + i];
+      const float keep = up ? v[half + i] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = LPR / (2 * G); off >= 1; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+  // lane owns head h = sum over levels k of (lane bit LPR/2^k set ? G/2^k : 0)
+  const int base = lane & ~(LPR - 1);
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    int src = base;
+#pragma unroll
+    for (int k = 1, off = LPR / 2; (G >> k) > 0; ++k, off >>= 1)
+      if (g & (G >> k)) src |= off;
+    x[g] = __shfl_sync(0xffffffffu, v[0], src);
+  }
+}
+
 // LPR lanes share a cached row; ST stages of kDecRows rows are in flight per CTA.
 template <int D, int LPR, int ST>
 struct DecPlan {
@@ -180,11 +219,9 @@ __global__ void __launch_bounds__(kDecThreads, DecPlan<D, LPR, ST>::kMinBlocks)
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int e = 0; e < 4 * NV; ++e) acc = __ffma2_rn(q[g][e], kf[e], acc);
-        float x = acc.x + acc.y;
-#pragma unroll
-        for (int off = 1; off < LPR; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        sc[g] = x;
+        sc[g] = acc.x + acc.y;
       }
+      reduce_heads<G, LPR>(sc, lane);
       if (valid) {
         float2 vf[4 * NV];
 #pragma unroll
