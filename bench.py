@@ -399,6 +399,9 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(3):
             pre()
         n_pre = 20
+        # a GPU-side sleep first, so the host has queued all calls before the GPU
+        # reaches them and the events time the kernels, not the Python call rate
+        torch.cuda._sleep(50_000_000)
         e0.record(stream)
         for _ in range(n_pre):
             pre()

@@ -602,7 +602,7 @@ namespace {
 bool pre_shape_ok(int P, int C, int heads) {
   if (P < 0 || heads < 1 || C < 1 || C % heads) return false;
   const int D = C / heads;
-  return (D == 64 || D == 128) && C % 256 == 0 && C <= 2048;
+  return (D == 64 || D == 128) && C % 256 == 0 && C <= 2048;  // C % 128: whole feature tiles
 }
 
 swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
@@ -614,7 +614,7 @@ swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, con
   if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
   PreParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!encode_2d_sw128(&p.tm_a, xn_ws, C, P, 128) || !encode_2d_sw128(&p.tm_b, w_qkv, C, 3LL * C, 256))
+  if (!encode_2d_sw128(&p.tm_a, xn_ws, C, P, 128) || !encode_2d_sw128(&p.tm_b, w_qkv, C, 3LL * C, 128))
     return SWA_ERR_CUDA;
   p.b_qkv = b_qkv;
   p.qn_w = qn_w;

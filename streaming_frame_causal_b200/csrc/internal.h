@@ -122,7 +122,7 @@ bool encode_2d_sw128(CUtensorMap* m, const void* base, int64_t inner, int64_t ro
 // ---------------------------------------------------------------- attn_pre prologue
 struct PreParams {
   CUtensorMap tm_a;     // norm1 output [P, C] bf16, box 64 x 128
-  CUtensorMap tm_b;     // w_qkv [3C, C] bf16, box 64 x 256
+  CUtensorMap tm_b;     // w_qkv [3C, C] bf16, box 64 x 128
   const float* b_qkv;   // [3C]
   const float* qn_w;    // [D] q_norm weight / bias
   const float* qn_b;

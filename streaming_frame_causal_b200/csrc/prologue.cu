@@ -5,7 +5,7 @@
 //   ln_rows_kernel   norm1: LayerNorm over C of each token, bf16 out
 //   qkv_pre_kernel   qkv = norm1(x) @ w_qkv^T + b_qkv on the tensor cores
 //                    (tcgen05, TMA-fed 4-stage ring, accumulator in TMEM), and
-//                    in the epilogue, per 128-token x 256-feature tile: the bias,
+//                    in the epilogue, per 128-token x 128-feature tile: the bias,
 //                    per-head LayerNorm of the q and k sections, RoPE on q and k
 //                    (the (2i, 2i+1) pairs times the caller's complex table: the
 //                    I/O page's complex-valued 3-D RoPE format), bf16 stores.
@@ -49,12 +49,18 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
   constexpr int kMaxChunks = 8;  // C <= 2048
   const int nch = C / 256;       // 8-element chunks per lane
   const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * C;
+  // all of the row's loads are issued before any is used (no early exit in the
+  // loop, so the unrolled loads are independent)
+  uint4 raw[kMaxChunks];
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c)
+    raw[c] = (c < nch) ? *reinterpret_cast<const uint4*>(xr + (c * 32 + lane) * 8) : make_uint4(0, 0, 0, 0);
   float v[kMaxChunks * 8];
   float s = 0.f;
 #pragma unroll
   for (int c = 0; c < kMaxChunks; ++c) {
     if (c >= nch) break;
-    const uint4 u = *reinterpret_cast<const uint4*>(xr + (c * 32 + lane) * 8);
+    const uint4 u = raw[c];
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -84,11 +90,17 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
   for (int c = 0; c < kMaxChunks; ++c) {
     if (c >= nch) break;
     const int col = (c * 32 + lane) * 8;
+    const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + col));
+    const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + col + 4));
+    const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + col));
+    const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + col + 4));
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float a0 = (v[c * 8 + 2 * e] - mean) * rs * __ldg(w + col + 2 * e) + __ldg(b + col + 2 * e);
-      const float a1 = (v[c * 8 + 2 * e + 1] - mean) * rs * __ldg(w + col + 2 * e + 1) + __ldg(b + col + 2 * e + 1);
+      const float a0 = (v[c * 8 + 2 * e] - mean) * rs * wv[2 * e] + bv[2 * e];
+      const float a1 = (v[c * 8 + 2 * e + 1] - mean) * rs * wv[2 * e + 1] + bv[2 * e + 1];
       o[e] = pack_bf16x2(a0, a1);
     }
     *reinterpret_cast<uint4*>(orow + col) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -98,16 +110,17 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
 // ---------------------------------------------------------------- qkv GEMM
 constexpr int kPreThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
 constexpr int kPreM = 128;        // tokens per tile
-constexpr int kPreN = 256;        // output features per tile
-constexpr int kPreStages = 4;
+constexpr int kPreN = 128;        // output features per tile (2 heads of 64 or 1 of 128)
+constexpr int kPreStages = 3;     // 96 KB of ring: two CTAs per SM, one's epilogue overlaps
+                                  // the other's main loop
 constexpr int kPreABytes = kPreM * 64 * 2;  // 16 KB: 128 rows x 64 columns
-constexpr int kPreBBytes = kPreN * 64 * 2;  // 32 KB
+constexpr int kPreBBytes = kPreN * 64 * 2;  // 16 KB
 constexpr int kPreStageBytes = kPreABytes + kPreBBytes;
 constexpr int kPreOffBar = kPreStages * kPreStageBytes;
 constexpr int kPreSmem = kPreOffBar + (2 * kPreStages + 1) * 8 + 16 + 1024;
 
 template <int D>
-__global__ void __launch_bounds__(kPreThreads, 1) qkv_pre_kernel(const __grid_constant__ PreParams p) {
+__global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_constant__ PreParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -193,53 +206,88 @@ __global__ void __launch_bounds__(kPreThreads, 1) qkv_pre_kernel(const __grid_co
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
       const float* nw = sec == 0 ? p.qn_w : p.kn_w;
       const float* nb = sec == 0 ? p.qn_b : p.kn_b;
+
+      // load 32 columns of this thread's row (+ bias) from TMEM
+      auto load32 = [&](int hh, int c0, float* v) {
+        __syncwarp();  // tcgen05.ld is warp-collective: all lanes converged
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + hh * D + c0, a);
+        tmem_wait_ld();
+        const float* bias = p.b_qkv + n0 + hh * D + c0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 bb = __ldg(reinterpret_cast<const float4*>(bias + j));
+          v[j] = __uint_as_float(a[j]) + bb.x;
+          v[j + 1] = __uint_as_float(a[j + 1]) + bb.y;
+          v[j + 2] = __uint_as_float(a[j + 2]) + bb.z;
+          v[j + 3] = __uint_as_float(a[j + 3]) + bb.w;
+        }
+      };
 #pragma unroll 1
       for (int hh = 0; hh < kPreN / D; ++hh) {
-        __syncwarp();  // tcgen05.ld is warp-collective: all lanes converged
-        uint32_t a[D];
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(tmem + lane_off + hh * D + c0, a + c0);
-        tmem_wait_ld();
-        if (row < p.P) {
-        const int fcol = n0 + hh * D;  // first output feature of this head
-        float v[D];
-#pragma unroll
-        for (int j = 0; j < D; ++j) v[j] = __uint_as_float(a[j]) + __ldg(p.b_qkv + fcol + j);
-        if (sec < 2) {
-          float s = 0.f;
-#pragma unroll
-          for (int j = 0; j < D; ++j) s += v[j];
-          const float mean = s / D;
-          float q = 0.f;
-#pragma unroll
-          for (int j = 0; j < D; ++j) q += (v[j] - mean) * (v[j] - mean);
-          const float rs = rsqrtf(q / D + p.eps);
-#pragma unroll
-          for (int j = 0; j < D; ++j) v[j] = (v[j] - mean) * rs * __ldg(nw + j) + __ldg(nb + j);
-          const float2* rt = reinterpret_cast<const float2*>(p.rot) + static_cast<int64_t>(row) * (D / 2);
-#pragma unroll
-          for (int i = 0; i < D / 2; ++i) {
-            const float2 cs = __ldg(rt + i);
-            const float x0 = v[2 * i], x1 = v[2 * i + 1];
-            v[2 * i] = x0 * cs.x - x1 * cs.y;
-            v[2 * i + 1] = x0 * cs.y + x1 * cs.x;
-          }
-        }
+        const bool valid = row < p.P;
         const int h = h0 + hh;
         uint8_t* dst;
         if (sec == 0)
-          dst = reinterpret_cast<uint8_t*>(p.q_out) + (static_cast<int64_t>(row) * p.H + h) * D * 2;
+          dst = reinterpret_cast<uint8_t*>(p.q_out) + (static_cast<int64_t>(valid ? row : 0) * p.H + h) * D * 2;
         else
-          dst = (sec == 1 ? p.k_dst : p.v_dst) + static_cast<int64_t>(row) * p.kv_row_bytes + h * D * 2;
+          dst = (sec == 1 ? p.k_dst : p.v_dst) + static_cast<int64_t>(valid ? row : 0) * p.kv_row_bytes + h * D * 2;
+        // q and k: LayerNorm statistics of the head first (sum and sum of squares)
+        float mean = 0.f, rs = 1.f;
+        if (sec < 2) {
+          float s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float v[32];
+            load32(hh, c0, v);
 #pragma unroll
-        for (int j = 0; j < D; j += 8) {
-          uint4 u;
-          u.x = pack_bf16x2(v[j], v[j + 1]);
-          u.y = pack_bf16x2(v[j + 2], v[j + 3]);
-          u.z = pack_bf16x2(v[j + 4], v[j + 5]);
-          u.w = pack_bf16x2(v[j + 6], v[j + 7]);
-          *reinterpret_cast<uint4*>(dst + j * 2) = u;
+            for (int j = 0; j < 32; ++j) {
+              s1 += v[j];
+              s2 += v[j] * v[j];
+            }
+          }
+          mean = s1 / D;
+          rs = rsqrtf(fmaxf(s2 / D - mean * mean, 0.f) + p.eps);
         }
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          load32(hh, c0, v);
+          if (sec < 2) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 ww = __ldg(reinterpret_cast<const float4*>(nw + c0 + j));
+              const float4 bb = __ldg(reinterpret_cast<const float4*>(nb + c0 + j));
+              v[j] = (v[j] - mean) * rs * ww.x + bb.x;
+              v[j + 1] = (v[j + 1] - mean) * rs * ww.y + bb.y;
+              v[j + 2] = (v[j + 2] - mean) * rs * ww.z + bb.z;
+              v[j + 3] = (v[j + 3] - mean) * rs * ww.w + bb.w;
+            }
+            if (valid) {
+              // RoPE: pairs (2i, 2i+1) times (cos, sin) of pair i; two pairs per 16-byte load
+              const float4* rt = reinterpret_cast<const float4*>(p.rot + static_cast<int64_t>(row) * D + c0);
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                const float4 cs = __ldg(rt + j / 4);
+                const float x0 = v[j], x1 = v[j + 1], x2 = v[j + 2], x3 = v[j + 3];
+                v[j] = x0 * cs.x - x1 * cs.y;
+                v[j + 1] = x0 * cs.y + x1 * cs.x;
+                v[j + 2] = x2 * cs.z - x3 * cs.w;
+                v[j + 3] = x2 * cs.w + x3 * cs.z;
+              }
+            }
+          }
+          if (valid) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 u;
+              u.x = pack_bf16x2(v[j], v[j + 1]);
+              u.y = pack_bf16x2(v[j + 2], v[j + 3]);
+              u.z = pack_bf16x2(v[j + 4], v[j + 5]);
+              u.w = pack_bf16x2(v[j + 6], v[j + 7]);
+              *reinterpret_cast<uint4*>(dst + (c0 + j) * 2) = u;
+            }
+          }
         }
       }
     }
