@@ -446,3 +446,39 @@ def attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads: in
     k = layer_norm(qkv[:, 1], kn_w, kn_b, eps)
     v = qkv[:, 2]
     return rope_complex(q, rot), rope_complex(k, rot), v.copy()
+
+
+# ----------------------------------------------------------------------------
+# 3-D RoPE table of a streaming frame ([IO] 3-D RoPE: complex-valued positions
+# [1, 1, S_global*P, head_dim/2] from WanRotaryPosEmbed, built internally when
+# enable_3d_rope=True)
+# ----------------------------------------------------------------------------
+def rope3d_bands(head_dim: int):
+    """Complex pairs per axis (t, h, w): the head's D/2 pairs split as
+    h = w = floor(D/6) pairs each and t = the rest (the Wan-style split of
+    head_dim into temporal, height and width parts)."""
+    d6 = head_dim // 6
+    n_h = n_w = d6
+    n_t = head_dim // 2 - n_h - n_w
+    return n_t, n_h, n_w
+
+
+def rope3d_table(frame_idx: int, P: int, num_special: int, grid_w: int, head_dim: int,
+                 theta: float = 10000.0) -> np.ndarray:
+    """(cos, sin) table [P, D/2, 2] of one frame.  Token k of the frame sits at
+    (t, h, w) = (frame_idx, (k - s) // grid_w, (k - s) % grid_w) for patch tokens
+    (k >= s = num_special) and at (frame_idx, 0, 0) for special tokens.  Pair j of
+    an axis band with n pairs rotates by pos * theta^(-j / n)."""
+    n_t, n_h, n_w = rope3d_bands(head_dim)
+    ang = np.zeros((P, head_dim // 2), dtype=np.float64)
+    for k in range(P):
+        if k < num_special:
+            t, h, w = frame_idx, 0, 0
+        else:
+            t, h, w = frame_idx, (k - num_special) // grid_w, (k - num_special) % grid_w
+        off = 0
+        for pos, n in ((t, n_t), (h, n_h), (w, n_w)):
+            for j in range(n):
+                ang[k, off + j] = pos * theta ** (-j / n)
+            off += n
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1)

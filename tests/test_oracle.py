@@ -553,3 +553,46 @@ def test_attn_pre_head_norms_closed_form():
     for t, out in ((0, q), (1, k)):
         s2 = lin[:, t].var(axis=-1)
         np.testing.assert_allclose((out ** 2).sum(axis=-1), D * s2 / (s2 + eps), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- 3-D RoPE table
+def test_rope3d_bands_split_head_dim():
+    assert orc.rope3d_bands(64) == (12, 10, 10)
+    assert orc.rope3d_bands(128) == (22, 21, 21)
+    assert orc.rope3d_bands(12) == (2, 2, 2)
+
+
+def test_rope3d_table_hand_worked_entry():
+    """head_dim 12: bands of 2 pairs each, frequencies 1 and theta^(-1/2) = 0.01.
+    Patch token 5 + 7 of a grid 3 wide sits at (t, h, w) = (4, 2, 1)."""
+    tab = orc.rope3d_table(frame_idx=4, P=20, num_special=5, grid_w=3, head_dim=12, theta=10000.0)
+    want_ang = [4.0, 0.04, 2.0, 0.02, 1.0, 0.01]
+    np.testing.assert_allclose(tab[12, :, 0], np.cos(want_ang), atol=1e-15)
+    np.testing.assert_allclose(tab[12, :, 1], np.sin(want_ang), atol=1e-15)
+
+
+def test_rope3d_table_structure():
+    D, P, s, gw = 64, 5 + 37 * 27, 5, 27
+    tab = orc.rope3d_table(frame_idx=9, P=P, num_special=s, grid_w=gw, head_dim=D)
+    np.testing.assert_allclose(np.hypot(tab[..., 0], tab[..., 1]), 1.0, atol=1e-14)
+    n_t, n_h, n_w = orc.rope3d_bands(D)
+    # special tokens: only the temporal band rotates
+    np.testing.assert_array_equal(tab[:s, n_t:, 0], 1.0)
+    np.testing.assert_array_equal(tab[:s, n_t:, 1], 0.0)
+    # every token of a frame shares the temporal band
+    np.testing.assert_array_equal(tab[:, :n_t], np.broadcast_to(tab[:1, :n_t], tab[:, :n_t].shape))
+
+
+def test_rope3d_rotated_dot_depends_on_displacement_only():
+    """q at token a of frame f1 and k at token b of frame f2: the rotated dot
+    product depends on (f2 - f1, h_b - h_a, w_b - w_a) only."""
+    D, s, gw = 64, 5, 27
+    g = np.random.default_rng(4)
+    q, k = g.standard_normal((1, 1, D)), g.standard_normal((1, 1, D))
+    def dot(f1, a, f2, b):
+        t1 = orc.rope3d_table(f1, a + 1, s, gw, D)[a:a + 1]
+        t2 = orc.rope3d_table(f2, b + 1, s, gw, D)[b:b + 1]
+        return np.sum(orc.rope_complex(q, t1) * orc.rope_complex(k, t2))
+    # token s + 28 is at (h, w) = (1, 1); s + 56 at (2, 2); s + 0 at (0, 0); s + 28 + 1 at (1, 2)
+    assert dot(3, s + 0, 5, s + 28) == pytest.approx(dot(10, s + 28, 12, s + 56), abs=1e-10)
+    assert dot(0, s + 1, 0, s + 29) == pytest.approx(dot(7, s + 28, 7, s + 56), abs=1e-10)
