@@ -213,6 +213,20 @@ swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_
                                        const float* kn_w, const float* kn_b, const float* rot, float eps,
                                        void* xn_ws, void* q_out, void* stream);
 
+/* 3-D RoPE table of one streaming frame, the rotation input of swa_attn_pre (the
+ * I/O page's 3-D RoPE: complex-valued positions [.., S_global*P, head_dim/2]
+ * from WanRotaryPosEmbed, generated internally when enable_3d_rope is set).
+ * Readings: token k of frame ``frame_idx`` sits at (t, h, w) = (frame_idx,
+ * (k - num_special) / grid_w, (k - num_special) % grid_w) for patch tokens and
+ * (frame_idx, 0, 0) for the num_special special tokens; the head_dim/2 pairs
+ * split into bands t | h | w of (head_dim/2 - 2*(head_dim/6), head_dim/6,
+ * head_dim/6) pairs; pair j of a band of n pairs turns by pos * theta^(-j/n).
+ * rot_out [P, head_dim/2, 2] f32 (cos, sin), device, 16-byte aligned.  Errors:
+ * SWA_ERR_ARG (negative index or size, num_special > P, grid_w < 1, odd or
+ * small head_dim, theta <= 1, null or misaligned output). */
+swa_status swa_rope3d_table(int frame_idx, int P, int num_special, int grid_w, int head_dim, double theta,
+                            float* rot_out, void* stream);
+
 /* Layout of one layer's metadata block, in int32 units. */
 typedef struct swa_meta_layout {
     int n_ints;          /* size of the block                                  */

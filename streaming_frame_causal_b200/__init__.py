@@ -67,6 +67,7 @@ _sigs = {
     "swa_stream_attend_transient": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "swa_attn_pre": (_i, [_vp] * 10 + [_i, _i, _i, C.c_float] + [_vp] * 5),
     "swa_stream_append_evict_pre": (_i, [_vp, _i, _i] + [_vp] * 10 + [C.c_float] + [_vp] * 3),
+    "swa_rope3d_table": (_i, [_i, _i, _i, _i, _i, C.c_double, _vp, _vp]),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
     "swa_stream_get_meta": (_i, [_vp, _i, _vp, _sz, _vp]),
     "swa_stream_k_storage": (_vp, [_vp, _i]),
@@ -178,6 +179,16 @@ def swa_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads
                              _ptr(kn_w), _ptr(kn_b), _ptr(rot), P, Cdim, heads, float(eps), _ptr(xn_ws),
                              _ptr(q_out), _ptr(k_out), _ptr(v_out), _stream(stream)), "swa_attn_pre")
     return q_out, k_out, v_out
+
+
+def swa_rope3d_table(frame_idx: int, P: int, num_special: int, grid_w: int, head_dim: int,
+                     theta: float = 10000.0, out=None, device="cuda", stream=None) -> torch.Tensor:
+    """3-D RoPE table [P, head_dim/2, 2] (cos, sin) of one streaming frame, the
+    ``rot`` input of swa_attn_pre (layout and readings: include/swa.h)."""
+    out = torch.empty(P, head_dim // 2, 2, dtype=torch.float32, device=device) if out is None else out
+    _check(_lib.swa_rope3d_table(frame_idx, P, num_special, grid_w, head_dim, float(theta), _ptr(out),
+                                 _stream(stream)), "swa_rope3d_table")
+    return out
 
 
 def swa_band_prefill(q, k, v, out, window: int, stream=None) -> torch.Tensor:

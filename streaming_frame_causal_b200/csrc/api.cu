@@ -650,6 +650,17 @@ extern "C" swa_status swa_attn_pre(const void* x, const float* ln_w, const float
                       static_cast<uint8_t*>(k_out), static_cast<uint8_t*>(v_out), static_cast<cudaStream_t>(stream));
 }
 
+extern "C" swa_status swa_rope3d_table(int frame_idx, int P, int num_special, int grid_w, int head_dim,
+                                       double theta, float* rot_out, void* stream) {
+  if (frame_idx < 0 || P < 0 || num_special < 0 || num_special > P || grid_w < 1 || head_dim < 6 ||
+      head_dim % 2 || !(theta > 1.0))
+    return SWA_ERR_ARG;
+  if (P == 0) return SWA_OK;
+  if (!rot_out || !aligned16(rot_out)) return SWA_ERR_ARG;
+  return cuda_status(launch_rope3d_table(rot_out, frame_idx, P, num_special, grid_w, head_dim, theta,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
                                                   const float* ln_w, const float* ln_b, const void* w_qkv,
                                                   const float* b_qkv, const float* qn_w, const float* qn_b,

@@ -140,6 +140,8 @@ struct PreParams {
 cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
                            cudaStream_t stream);
 cudaError_t launch_qkv_pre(const PreParams& p, cudaStream_t stream);
+cudaError_t launch_rope3d_table(float* rot, int frame, int P, int num_special, int grid_w, int head_dim,
+                                double theta, cudaStream_t stream);
 int decode_chunks(int B, int Hkv, int W);
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);

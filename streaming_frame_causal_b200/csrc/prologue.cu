@@ -301,6 +301,35 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
   }
 }
 
+// ---------------------------------------------------------------- 3-D RoPE table
+// One thread per (token, pair): token k of frame t sits at (t, h, w) = (t,
+// (k - s) / grid_w, (k - s) % grid_w) for patch tokens, (t, 0, 0) for the s
+// special tokens; pair j of an axis band of n pairs turns by pos * theta^(-j/n).
+// The bands split the head_dim/2 pairs as t | h | w with h = w = head_dim / 6
+// pairs (the I/O page's 3-D RoPE, WanRotaryPosEmbed).  Angles in double so the
+// table does not lose accuracy at large frame indices.
+__global__ void rope3d_table_kernel(float* __restrict__ rot, int frame, int P, int ns, int grid_w, int half,
+                                    int n_t, int n_h, double log_theta) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(P) * half) return;
+  const int k = static_cast<int>(idx / half);
+  const int j = static_cast<int>(idx - static_cast<int64_t>(k) * half);
+  const int h = k < ns ? 0 : (k - ns) / grid_w;
+  const int w = k < ns ? 0 : (k - ns) % grid_w;
+  int pos, jj, n;
+  if (j < n_t) {
+    pos = frame; jj = j; n = n_t;
+  } else if (j < n_t + n_h) {
+    pos = h; jj = j - n_t; n = n_h;
+  } else {
+    pos = w; jj = j - n_t - n_h; n = half - n_t - n_h;
+  }
+  const double ang = static_cast<double>(pos) * exp(-log_theta * jj / n);
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  reinterpret_cast<float2*>(rot)[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+}
+
 template <int D>
 cudaError_t launch_pre_d(const PreParams& p, cudaStream_t stream) {
   static int attr_dev_mask = 0;
@@ -326,6 +355,19 @@ cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* 
   if (P <= 0) return cudaSuccess;
   ln_rows_kernel<<<cdiv(P, 8), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), w, b,
                                                   static_cast<__nv_bfloat16*>(out), P, C, eps);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope3d_table(float* rot, int frame, int P, int num_special, int grid_w, int head_dim,
+                                double theta, cudaStream_t stream) {
+  const int half = head_dim / 2;
+  const int n_h = head_dim / 6;
+  const int n_t = half - 2 * n_h;
+  const int64_t n = static_cast<int64_t>(P) * half;
+  if (n <= 0) return cudaSuccess;
+  rope3d_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+      rot, frame, P, num_special, grid_w, half, n_t, n_h, std::log(theta));
   count_launches(1);
   return cudaGetLastError();
 }

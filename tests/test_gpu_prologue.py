@@ -92,3 +92,39 @@ def test_fused_append_writes_the_prologue_into_the_slot(swa, special):
             sp0 = cache.layout.n_slots * ppf * 16 + (j - S) * 5
             assert torch.equal(ks[sp0:sp0 + 5], frames_k[j][:5])
     assert swa.swa_device_error_check() == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope3d_table_matches_oracle(swa, D):
+    """The lingbot-map frame (5 special tokens + a 37 x 27 patch grid) at frames
+    0, 7 and 999: angles in double on the device, stored as f32."""
+    P, s, gw = 5 + 37 * 27, 5, 27
+    for f in (0, 7, 999):
+        got = swa.swa_rope3d_table(f, P, s, gw, D).cpu().numpy()
+        ref = orc.rope3d_table(f, P, s, gw, D)
+        np.testing.assert_allclose(got, ref, atol=2e-7, rtol=0)
+
+
+def test_prologue_with_3d_rope_table(swa):
+    P, C, H = 5 + 37 * 27, 1024, 16
+    inp = synth.prologue_inputs(seed=77, P=P, C=C, heads=H)
+    d = {k: v.cuda() for k, v in inp.items()}
+    rot = swa.swa_rope3d_table(42, P, 5, 27, C // H)
+    q, k, v = swa.swa_attn_pre(d["x"], *(d[n] for n in ORDER[:-1]), rot, heads=H, eps=EPS)
+    torch.cuda.synchronize()
+    a = {n: t.double().numpy() for n, t in inp.items()}
+    a["rot"] = orc.rope3d_table(42, P, 5, 27, C // H)
+    rq, rk, rv = orc.attn_pre(a["x"], *(a[n] for n in ORDER), heads=H, eps=EPS)
+    for got, ref, name in ((q, rq, "q"), (k, rk, "k"), (v, rv, "v")):
+        check_bf16(got.float().cpu().numpy(), ref, f"{name} with the 3-D table")
+
+
+def test_rope3d_table_rejects_bad_arguments(swa):
+    lib = swa._lib
+    buf = torch.empty(16, 32, 2, device="cuda")
+    assert lib.swa_rope3d_table(-1, 16, 5, 3, 64, 10000.0, buf.data_ptr(), None) == -1
+    assert lib.swa_rope3d_table(0, 16, 17, 3, 64, 10000.0, buf.data_ptr(), None) == -1
+    assert lib.swa_rope3d_table(0, 16, 5, 0, 64, 10000.0, buf.data_ptr(), None) == -1
+    assert lib.swa_rope3d_table(0, 16, 5, 3, 63, 10000.0, buf.data_ptr(), None) == -1
+    assert lib.swa_rope3d_table(0, 16, 5, 3, 64, 1.0, buf.data_ptr(), None) == -1
+    assert lib.swa_rope3d_table(0, 16, 5, 3, 64, 10000.0, None, None) == -1
