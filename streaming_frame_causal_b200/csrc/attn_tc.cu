@@ -20,9 +20,12 @@
 // whole 128-column row of S in registers.
 // The two query tiles ping-pong: while softmax A turns S_A into P_A, the tensor
 // core runs P_B V and Q_B K^T, and the other way round.  S (f32, 128 columns),
-// P (bf16 pairs, 64 columns) and O (f32, D columns) of each tile live in tensor
-// memory; P feeds the PV product straight from TMEM (A operand), so the only
-// shared-memory operands are Q, K and V, staged by TMA with 128-byte swizzle.
+// P (bf16 pairs, 64 columns written over the front of S once it is read) and O
+// (f32, D columns, plus the row-sum column at head_dim 64) of each tile live in
+// tensor memory; P feeds the PV product straight from TMEM (A operand), so the
+// shared-memory operands are Q, K and V, staged by TMA with 128-byte swizzle
+// (and at head_dim 64 a constant block that turns one PV column into the row
+// sum).
 // Online softmax uses exp2 with the scale folded in and skips rescaling O
 // unless the running maximum grows by more than 2^8 (exact after the final
 // division by the row sum).
