@@ -9,10 +9,11 @@
 // the cache; sliding-window explainer: token band t-W+1..t).
 //
 // CTA organisation (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer: Q tiles once, then K key tiles into a ring
+//   warp 0      TMA producer: Q tiles once, then K key tiles into a ring (and
+//               at head_dim 64 the V tile of the same key tile beside it)
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
 //   warp 2      idle
-//   warp 3      TMA producer: V key tiles into a second ring
+//   warp 3      TMA producer at head_dim 128: V key tiles into a second ring
 //   warps 4-7   softmax for query tile A (one thread per query row)
 //   warps 8-11  softmax for query tile B
 // After set-up, warpgroup 0 gives registers back (setmaxnreg.dec to 64) and the
@@ -65,6 +66,11 @@ struct Plan {
   // then has N = D + 16.  At D = 128 that would not fit tensor memory; the
   // softmax threads add the row sums themselves.
   static constexpr bool kSumCol = (D == 64);
+  // K and V stages with their own barriers (released after the QK^T and after
+  // the PV respectively) for the two-stage ring at head_dim 128; one barrier per
+  // stage for both at head_dim 64, where the four-stage ring has slack and the
+  // single MMA-issuing thread saves a wait and a commit per key tile
+  static constexpr bool kSplitKV = (D == 128);
   static constexpr int kON = kSumCol ? D + 16 : D;  // O columns written by the PV
   // Tensor-memory columns: S 2x128 | O 2x128 (D or D + 16 used).  P (64 columns
   // of bf16 pairs) reuses the first half of its own S once the softmax has read
@@ -301,11 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   reg_dealloc<kRegsCtl>();
   if (warp == 0 || warp == 3) {
     // ------------------------------------------------------------ producers
-    // lane 0 of warp 0 loads the Q tiles and the K ring, lane 0 of warp 3 the V ring
+    // lane 0 of warp 0 loads the Q tiles and the K ring, lane 0 of warp 3 the V
+    // ring (split K/V barriers); without the split warp 0 loads both
     const bool is_k = (warp == 0);
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && T > 0 && (PL::kSplitKV || is_k)) {
       const CUtensorMap* tm = is_k ? &p.tm_k : &p.tm_v;
       tma_prefetch_desc(tm);
+      if (!PL::kSplitKV) tma_prefetch_desc(&p.tm_v);
       if (is_k) {
         tma_prefetch_desc(&p.tm_q);
         for (int g = 0; g < (has_b ? 2 : 1); ++g) {
@@ -335,9 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         int krow, kvalid;
         cursor_tile(w, cur, &krow, &kvalid);
-        mbar_arrive_expect_tx(full, PL::kTileBytes);
-        for (int sub = 0; sub < PL::kSubs; ++sub)
+        mbar_arrive_expect_tx(full, PL::kSplitKV ? PL::kTileBytes : 2 * PL::kTileBytes);
+        for (int sub = 0; sub < PL::kSubs; ++sub) {
           tma_load_4d(ring + st * PL::kTileBytes + sub * kSubBytes, tm, full, sub * 64, w.kvh, krow, w.b);
+          if (!PL::kSplitKV)
+            tma_load_4d(base + PL::kOffV + st * PL::kTileBytes + sub * kSubBytes, &p.tm_v, full, sub * 64, w.kvh,
+                        krow, w.b);
+        }
         cursor_next(w, cur);
         ++issued;
       }
@@ -395,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           issue_qk(1, 0);
           mma_commit(s_full(1));
         }
-        mma_commit(k_empty(0));
+        if (PL::kSplitKV) mma_commit(k_empty(0));
       }
       const int ng = has_b ? 2 : 1;
       // Fixed order per key tile: PV_A(j) QK_A(j+1) | PV_B(j) QK_B(j+1), each
@@ -407,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int st1 = (j + 1) % PL::kStages;
         const bool more = j + 1 < T;
         if (more && !mbar_wait(k_full(st1), ((j + 1) / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
-        if (!mbar_wait(v_full(st), (j / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+        if (PL::kSplitKV && !mbar_wait(v_full(st), (j / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
 #pragma unroll 1
         for (int g = 0; g < ng; ++g) {
           if (!mbar_wait(p_full(g), j & 1, p.err, ERR_WAIT_MMA)) {
@@ -424,8 +436,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
         if (!ok) break;
-        mma_commit(v_empty(st));
-        if (more) mma_commit(k_empty(st1));
+        if (PL::kSplitKV) {
+          mma_commit(v_empty(st));
+          if (more) mma_commit(k_empty(st1));
+        } else {
+          mma_commit(k_empty(st));  // K_j and V_j leave together after PV_B(j)
+        }
       }
       // drain every MMA this thread issued before the CTA may free TMEM
       mma_commit(drain(0));
