@@ -120,6 +120,12 @@ bool swa::encode_2d_sw128(CUtensorMap* m, const void* base, int64_t inner, int64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool swa::encode_4d_sw128(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B) {
+  return make_map(m, base, D, H, N, B);
+}
+
+int swa::device_sms() { return num_sms(); }
+
 bool swa::encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;

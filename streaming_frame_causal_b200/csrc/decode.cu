@@ -436,8 +436,20 @@ cudaError_t launch_dec_pick(const DecodeParams& p, cudaStream_t stream) {
 }
 }  // namespace
 
+cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t stream) {
+  if (p.D == 128)
+    decode_combine_kernel<128><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
+  else if (p.D == 64)
+    decode_combine_kernel<64><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_bf16(const DecodeParams& p_in, cudaStream_t stream) {
   const int G = p_in.Hq / p_in.Hkv;
+  // head_dim 128: the tensor-core kernel (decode_tc.cu)
+  if (decode_tc_supported(p_in.D, G)) return launch_decode_tc(p_in, device_sms(), stream);
   DecodeParams p = p_in;
   // K/V caches viewed as rows [B*W, Hkv, D]; one box = 32 rows of one KV head
   if (!encode_rows_map(&p.tm_k, p.k_cache, p.D, p.Hkv, static_cast<int64_t>(p.B) * p.W, kDecRows) ||

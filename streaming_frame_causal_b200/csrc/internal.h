@@ -96,7 +96,8 @@ cudaError_t launch_transient_prepare(const TransientParams& p, cudaStream_t stre
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
   CUtensorMap tm_k;   // K cache as rows [B*W, Hkv, D], box = 32 rows x 1 head x D
-  CUtensorMap tm_v;
+  CUtensorMap tm_v;   // (tensor-core decode: [B, W, Hkv, D] as 4-D, box 64 x 1 x 128 x 1, 128-byte swizzle)
+  CUtensorMap tm_q;   // tensor-core decode: q as [B*Hq, D], box 64 x 16, 128-byte swizzle
   const void* q;      // [B, Hq, D]
   const void* k_new;  // [B, Hkv, D]
   const void* v_new;
@@ -112,6 +113,15 @@ struct DecodeParams {
 };
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
+// tensor-core decode (head_dim 128, G in {1, 2, 4, 8}): appends the new token,
+// runs the persistent kernel and the combine; p.chunks = partial slots available
+bool decode_tc_supported(int D, int G);
+int decode_tc_pieces(int B, int Hkv, int n_valid, int max_pieces, int sms);
+cudaError_t launch_decode_tc(const DecodeParams& p, int sms, cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t stream);
+// bf16 [B, N, H, D] as a 4-D map {D, H, N, B}, box 64 x 1 x 128 x 1, 128-byte swizzle
+bool encode_4d_sw128(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B);
+int device_sms();
 int decode_chunk_len(int n_valid, int chunks);
 // bf16 [rows, H, D] as a 3-D tensor map with a box of box_rows rows of one head (no swizzle)
 bool encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows);

@@ -43,6 +43,14 @@ def test_band_parity(swa, N, Hq, Hkv, D, W, dtype):
     (2, 64, 10, 8, 2, 128, torch.bfloat16),     # buffer not yet full
     (2, 96, 95, 4, 1, 64, torch.bfloat16),      # exactly full
     (2, 32, 40, 4, 2, 64, torch.float32),
+    # head_dim 128 on the tensor cores: one to eight query heads per KV head,
+    # a ragged last key tile, a partly filled window over several tiles, and a
+    # single KV head whose keys are cut into five pieces
+    (2, 300, 1000, 16, 16, 128, torch.bfloat16),
+    (4, 1024, 500, 16, 8, 128, torch.bfloat16),
+    (3, 256, 700, 64, 8, 128, torch.bfloat16),
+    (1, 640, 639, 8, 1, 128, torch.bfloat16),
+    (2, 130, 129, 4, 1, 128, torch.bfloat16),
 ])
 def test_decode_parity(swa, B, W, pos, Hq, Hkv, D, dtype):
     q, kn, vn, kc, vc = synth.decode_inputs(seed=pos, B=B, W=W, Hq=Hq, Hkv=Hkv, D=D, dtype=dtype)
