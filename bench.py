@@ -104,7 +104,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "attn": ("attn_tc.cu", "ptx.cuh", "tile_sched.h", "exp2_poly.cuh"),
-    "decode": ("decode.cu", "ptx.cuh"),
+    "decode": ("decode.cu", "decode_tc.cu", "ptx.cuh"),
 }
 
 
@@ -439,7 +439,7 @@ def run_ours(args, rank, world, local_rank):
             cands.append((share, per["stream"], "attn_tc_kernel<64> stream attend + append + combine, 8 frames",
                           stage_flops["stream"], "attn_tc_stream_72x1004_h16_d64", "tensor"))
     if "decode" in per:
-        cands.append((per["decode"], per["decode"], "decode_kernel<128,4> B64 W4096", decode_bytes(),
+        cands.append((per["decode"], per["decode"], "decode_tc_kernel<4> B64 W4096", decode_bytes(),
                       "decode_b64_w4096_gqa32_8_d128", "hbm"))
     _, kms, kname, kwork, tkey, bound = max(cands)
     if bound == "tensor":
