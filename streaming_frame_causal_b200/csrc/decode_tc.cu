@@ -1,5 +1,5 @@
 // decode_tc.cu -- GQA decode against the rolling KV cache on the tensor cores
-// (sm_100a), bf16 in, f32 accumulate, head_dim 128.
+// (sm_100a), bf16 in, f32 accumulate, head_dim 64 or 128.
 //
 // What it computes (sliding-window explainer, rolling-buffer decode): the new
 // token's G query heads of a KV group attend, with softmax(q k^T / sqrt(D)), to
@@ -9,7 +9,9 @@
 // Layout of the work.  With one query token there are only G <= 16 query rows
 // per (batch, KV head), so the products run with the keys as the M dimension:
 //   S^T[128 keys x 16] = K_tile[128 x D] . Q^T        (A = K, K-major; B = Q, K-major)
-//   O^T[D x 16]       += V_tile^T[D x 128] . P^T      (A = V, MN-major; B = P^T, K-major)
+//   O^T[128 x 16]     += V_tile^T[. x 128] . P^T      (A = V, MN-major; B = P^T, K-major)
+// (the second product always has M = 128; at head_dim 64 its rows 64..127 are
+// never read)
 // S^T lands in tensor memory with one key per lane, so the softmax is spread
 // over 128 threads (one key each, G scores per thread); the head-wise maximum
 // of a tile is a warp shuffle reduction plus an exchange between four warps.
@@ -41,24 +43,32 @@ namespace swa {
 namespace {
 
 constexpr int kTcdThreads = 192;
-constexpr int kTcdD = 128;          // head_dim
 constexpr int kTcdKeys = 128;       // keys per tile (M of the first product)
 constexpr int kTcdN = 16;           // query-head columns (N of both products; G <= 16 used)
-constexpr int kTcdStages = 3;       // K/V ring depth
 constexpr int kTcdSub = kTcdKeys * 128;           // one 64-column swizzled sub-tile of K or V: 16 KB
-constexpr int kTcdTile = 2 * kTcdSub;             // K (or V) tile: 32 KB
-constexpr int kTcdStage = 2 * kTcdTile;           // K + V: 64 KB
 constexpr int kTcdSmallSub = kTcdN * 128;         // Q or P^T sub-tile: 16 rows x 128 bytes
 constexpr int kTcdSmall = 2 * kTcdSmallSub;       // Q or P^T buffer: 4 KB
-constexpr int kOffQ = kTcdStages * kTcdStage;     // 2 Q buffers
-constexpr int kOffP = kOffQ + 2 * kTcdSmall;      // 2 P^T buffers
-constexpr int kOffRed = kOffP + 2 * kTcdSmall;    // [2][4][16] tile maxima, [4][16] row sums
-constexpr int kOffBar = kOffRed + 3 * 4 * kTcdN * 4;
-constexpr int kNumBars = 2 + 2 + 2 * kTcdStages + 2 + 2 + 2 + 3 + 1;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kTcdSmem = kOffTmemSlot + 16 + 1024;  // + alignment slack
 constexpr uint32_t kTcdTmemCols = 64;               // S^T 2 x 16 | O^T 16 (+ 16 unused)
-static_assert(kTcdSmem <= 227 * 1024, "shared memory");
+
+// Shared-memory plan per head_dim: the K/V ring, 2 Q and 2 P^T buffers, the
+// softmax exchange area, barriers.  At head_dim 64 a K or V tile is one
+// 64-column sub-tile and the ring is deeper (five 32 KB stages).
+template <int D>
+struct TcdPlan {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr int kSubs = D / 64;
+  static constexpr int kStages = (D == 64) ? 5 : 3;
+  static constexpr int kTile = kSubs * kTcdSub;       // K (or V) tile
+  static constexpr int kStage = 2 * kTile;            // K + V
+  static constexpr int kOffQ = kStages * kStage;      // 2 Q buffers
+  static constexpr int kOffP = kOffQ + 2 * kTcdSmall; // 2 P^T buffers
+  static constexpr int kOffRed = kOffP + 2 * kTcdSmall;  // [2][4][16] tile maxima, [4][16] row sums
+  static constexpr int kOffBar = kOffRed + 3 * 4 * kTcdN * 4;
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 3 + 1;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffTmemSlot + 16 + 1024;  // + alignment slack
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
 
 // kind::f16 instruction descriptor with A MN-major (transpose A, bit 15)
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kTcdN, 0);
@@ -93,9 +103,18 @@ SWA_DEV TcdUnit tcd_unit(const DecodeParams& p, int unit) {
   return u;
 }
 
-template <int G>
+template <int D, int G>
 __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
   static_assert(G >= 1 && G <= kTcdN, "query heads per KV head");
+  using PL = TcdPlan<D>;
+  constexpr int kTcdStages = PL::kStages;
+  constexpr int kTcdStage = PL::kStage;
+  constexpr int kTcdTile = PL::kTile;
+  constexpr int kOffQ = PL::kOffQ;
+  constexpr int kOffP = PL::kOffP;
+  constexpr int kOffRed = PL::kOffRed;
+  constexpr int kOffBar = PL::kOffBar;
+  constexpr int kOffTmemSlot = PL::kOffTmemSlot;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -162,8 +181,8 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(q_full(qb), kTcdSmall);
-        for (int sub = 0; sub < 2; ++sub)
+        mbar_arrive_expect_tx(q_full(qb), PL::kSubs * kTcdSmallSub);
+        for (int sub = 0; sub < PL::kSubs; ++sub)
           tma_load_2d(base + kOffQ + qb * kTcdSmall + sub * kTcdSmallSub, &p.tm_q, q_full(qb), sub * 64,
                       u.b * p.Hq + u.kvh * G);
         ++lu;
@@ -176,7 +195,7 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
           const int row = u.t_begin + j * kTcdKeys;
           const uint32_t dst = base + st * kTcdStage;
           mbar_arrive_expect_tx(kv_full(st), kTcdStage);
-          for (int sub = 0; sub < 2; ++sub) {
+          for (int sub = 0; sub < PL::kSubs; ++sub) {
             tma_load_4d(dst + sub * kTcdSub, &p.tm_k, kv_full(st), sub * 64, u.kvh, row, u.b);
             tma_load_4d(dst + kTcdTile + sub * kTcdSub, &p.tm_v, kv_full(st), sub * 64, u.kvh, row, u.b);
           }
@@ -192,7 +211,10 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint64_t dk0 = sdesc_sw128(base, 16, 1024);                    // K of stage 0 (A, K-major)
-      const uint64_t dv0 = sdesc_sw128(base + kTcdTile, kTcdSub, 1024);    // V of stage 0 (A, MN-major)
+      // V of stage 0 (A, MN-major): the second 64-row group of M is the second
+      // sub-tile at head_dim 128; at 64 it is the next 16 KB of shared memory
+      // (rows D..127 of O^T, never read)
+      const uint64_t dv0 = sdesc_sw128(base + kTcdTile, kTcdSub, 1024);
       const uint64_t dq0 = sdesc_sw128(base + kOffQ, 16, 1024);            // Q buffer 0 (B, K-major)
       const uint64_t dp0 = sdesc_sw128(base + kOffP, 16, 1024);            // P^T buffer 0 (B, K-major)
       constexpr uint64_t kStageStep = kTcdStage >> 4;
@@ -202,7 +224,7 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
         const uint64_t dq = dq0 + qb * kSmallStep;
         const uint32_t tS = tmem + (jj & 1) * kTcdN;
 #pragma unroll
-        for (int kk = 0; kk < kTcdD / 16; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tS, dk + (((kk >> 2) * kTcdSub + (kk & 3) * 32) >> 4),
                  dq + (((kk >> 2) * kTcdSmallSub + (kk & 3) * 32) >> 4), kIdescS, kk > 0 ? 1u : 0u);
       };
@@ -387,8 +409,10 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
       uint32_t ov[16];
       tmem_ld16(tO, ov);
       tmem_wait_ld();
+      if (r < D) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) p.part_o[(pbase + h) * kTcdD + r] = __uint_as_float(ov[h]);
+        for (int h = 0; h < G; ++h) p.part_o[(pbase + h) * D + r] = __uint_as_float(ov[h]);
+      }
       float* lsum = red + 2 * 4 * kTcdN;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -438,19 +462,20 @@ __global__ void decode_append_kernel(const DecodeParams p) {
   }
 }
 
-template <int G>
+template <int D, int G>
 cudaError_t launch_tcd(const DecodeParams& p, int grid, cudaStream_t stream) {
+  constexpr int kSmem = TcdPlan<D>::kSmem;
   static int attr_dev_mask = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const int bit = 1 << (dev & 31);
   if (!(attr_dev_mask & bit)) {
     const cudaError_t e =
-        cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcdSmem);
+        cudaFuncSetAttribute(decode_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_dev_mask |= bit;
   }
-  decode_tc_kernel<G><<<grid, kTcdThreads, kTcdSmem, stream>>>(p);
+  decode_tc_kernel<D, G><<<grid, kTcdThreads, kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -477,7 +502,7 @@ int decode_tc_pieces(int B, int Hkv, int n_valid, int max_pieces, int sms) {
   return best;
 }
 
-bool decode_tc_supported(int D, int G) { return D == kTcdD && (G == 1 || G == 2 || G == 4 || G == 8); }
+bool decode_tc_supported(int D, int G) { return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8); }
 
 // p.chunks on entry: the partial slots the workspace holds per (batch, KV head)
 cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t stream) {
@@ -496,11 +521,20 @@ cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t str
   decode_append_kernel<<<static_cast<int>(std::min<int64_t>(1024, (n16 + 255) / 256)), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  switch (G) {
-    case 1: e = launch_tcd<1>(p, grid, stream); break;
-    case 2: e = launch_tcd<2>(p, grid, stream); break;
-    case 4: e = launch_tcd<4>(p, grid, stream); break;
-    default: e = launch_tcd<8>(p, grid, stream); break;
+  if (p.D == 128) {
+    switch (G) {
+      case 1: e = launch_tcd<128, 1>(p, grid, stream); break;
+      case 2: e = launch_tcd<128, 2>(p, grid, stream); break;
+      case 4: e = launch_tcd<128, 4>(p, grid, stream); break;
+      default: e = launch_tcd<128, 8>(p, grid, stream); break;
+    }
+  } else {
+    switch (G) {
+      case 1: e = launch_tcd<64, 1>(p, grid, stream); break;
+      case 2: e = launch_tcd<64, 2>(p, grid, stream); break;
+      case 4: e = launch_tcd<64, 4>(p, grid, stream); break;
+      default: e = launch_tcd<64, 8>(p, grid, stream); break;
+    }
   }
   if (e != cudaSuccess) return e;
   e = launch_decode_combine(p, stream);

@@ -51,6 +51,9 @@ def test_band_parity(swa, N, Hq, Hkv, D, W, dtype):
     (3, 256, 700, 64, 8, 128, torch.bfloat16),
     (1, 640, 639, 8, 1, 128, torch.bfloat16),
     (2, 130, 129, 4, 1, 128, torch.bfloat16),
+    # head_dim 64 on the same kernel (one 64-column sub-tile per key tile)
+    (2, 700, 699, 8, 4, 64, torch.bfloat16),
+    (3, 300, 1000, 8, 8, 64, torch.bfloat16),
 ])
 def test_decode_parity(swa, B, W, pos, Hq, Hkv, D, dtype):
     q, kn, vn, kc, vc = synth.decode_inputs(seed=pos, B=B, W=W, Hq=Hq, Hkv=Hkv, D=D, dtype=dtype)
