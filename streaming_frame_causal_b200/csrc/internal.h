@@ -95,9 +95,9 @@ cudaError_t launch_transient_prepare(const TransientParams& p, cudaStream_t stre
 
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
-  CUtensorMap tm_k;   // K cache as rows [B*W, Hkv, D], box = 32 rows x 1 head x D
-  CUtensorMap tm_v;   // (tensor-core decode: [B, W, Hkv, D] as 4-D, box 64 x 1 x 128 x 1, 128-byte swizzle)
-  CUtensorMap tm_q;   // tensor-core decode: q as [B*Hq, D], box 64 x 16, 128-byte swizzle
+  CUtensorMap tm_k;   // K cache [B, W, Hkv, D] as 4-D, box 64 x 1 x 128 x 1, 128-byte swizzle
+  CUtensorMap tm_v;   // V cache, the same
+  CUtensorMap tm_q;   // q as [B*Hq, D], box 64 x 16, 128-byte swizzle
   const void* q;      // [B, Hq, D]
   const void* k_new;  // [B, Hkv, D]
   const void* v_new;
@@ -122,9 +122,6 @@ cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t stream);
 // bf16 [B, N, H, D] as a 4-D map {D, H, N, B}, box 64 x 1 x 128 x 1, 128-byte swizzle
 bool encode_4d_sw128(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B);
 int device_sms();
-int decode_chunk_len(int n_valid, int chunks);
-// bf16 [rows, H, D] as a 3-D tensor map with a box of box_rows rows of one head (no swizzle)
-bool encode_rows_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows, int box_rows);
 // bf16 matrix [rows, inner] (inner contiguous) as a 2-D map; box = 64 columns x
 // box_rows rows, 128-byte swizzle
 bool encode_2d_sw128(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int box_rows);
