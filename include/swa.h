@@ -85,6 +85,17 @@ int64_t swa_sched_prefill(int B, int S, int P, int heads, int sliding_window_siz
                           int num_frame_per_block, int num_frame_for_scale,
                           int32_t* out, int64_t cap);
 
+/* swa_sched_decode: the launch swa_decode makes for batch B, Hkv KV heads, a
+ * W-slot rolling cache and position ``pos`` on a GPU of ``sms`` SMs
+ * (sliding-window explainer, rolling buffer: the valid slots are min(pos+1, W)).
+ * Each (batch, KV head) cuts its valid slots into ``pieces`` pieces of
+ * ``piece_len`` slots (whole 128-key tiles; the last piece may be shorter or
+ * empty), at most ``slots`` = the partial slots the decode workspace holds; the
+ * units (batch, KV head, piece) go round-robin to ``grid`` persistent CTAs.
+ * out[5] = {pieces, piece_len, grid, slots, n_valid}.  Returns SWA_OK or
+ * SWA_ERR_ARG. */
+int swa_sched_decode(int B, int Hkv, int W, long long pos, int sms, int32_t* out);
+
 /* ---------------------------------------------------------------- prefill
  * Frame-causal sliding-window attention over a whole clip ([AGG], [IO]).
  *   q, k, v, out: [B, S*P, heads, head_dim] contiguous, i.e. the pages'

@@ -57,6 +57,7 @@ _sigs = {
     "swa_version": (_i, []),
     "swa_sched_frame_intervals": (_i, [_i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i)]),
     "swa_sched_prefill": (_i64, [_i, _i, _i, _i, _i, _i, _i, _vp, _i64]),
+    "swa_sched_decode": (_i, [_i, _i, _i, C.c_longlong, _i, _vp]),
     "swa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "swa_stream_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
     "swa_stream_create": (_i, [C.POINTER(_vp), C.POINTER(swa_stream_cfg), _vp, _sz, _vp]),
@@ -151,6 +152,13 @@ def swa_sched_prefill(B: int, S: int, P: int, heads: int, sliding_window_size: i
     _lib.swa_sched_prefill(B, S, P, heads, sliding_window_size, num_frame_per_block, num_frame_for_scale,
                            out.ctypes.data, n)
     return out
+
+
+def swa_sched_decode(B: int, Hkv: int, W: int, pos: int, sms: int = 148) -> dict:
+    """The decode's launch plan (see include/swa.h)."""
+    out = (C.c_int * 5)()
+    _check(_lib.swa_sched_decode(B, Hkv, W, pos, sms, out), "swa_sched_decode")
+    return {"pieces": out[0], "piece_len": out[1], "grid": out[2], "slots": out[3], "n_valid": out[4]}
 
 
 # ---------------------------------------------------------------- prefill

@@ -197,6 +197,19 @@ extern "C" int64_t swa_sched_prefill(int B, int S, int P, int heads, int sliding
   return n;
 }
 
+extern "C" int swa_sched_decode(int B, int Hkv, int W, long long pos, int sms, int32_t* out) {
+  if (B < 1 || Hkv < 1 || W < 1 || pos < 0 || sms < 1 || !out) return SWA_ERR_ARG;
+  const int n_valid = (pos >= W - 1) ? W : static_cast<int>(pos + 1);
+  const int slots = decode_chunks(B, Hkv, W);
+  const DecodeTcPlan pl = decode_tc_plan(B, Hkv, n_valid, slots, sms);
+  out[0] = pl.pieces;
+  out[1] = pl.piece_len;
+  out[2] = pl.grid;
+  out[3] = slots;
+  out[4] = n_valid;
+  return SWA_OK;
+}
+
 // ==================================================================== prefill
 extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, void* out, int B, int S, int P,
                                   int C, int heads, int head_dim, int sliding_window_size,

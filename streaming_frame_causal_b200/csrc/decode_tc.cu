@@ -502,6 +502,14 @@ int decode_tc_pieces(int B, int Hkv, int n_valid, int max_pieces, int sms) {
   return best;
 }
 
+DecodeTcPlan decode_tc_plan(int B, int Hkv, int n_valid, int max_pieces, int sms) {
+  DecodeTcPlan pl;
+  pl.pieces = decode_tc_pieces(B, Hkv, n_valid, max_pieces, sms);
+  pl.piece_len = cdiv(cdiv(n_valid, pl.pieces), kTcdKeys) * kTcdKeys;
+  pl.grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(B) * Hkv * pl.pieces, sms));
+  return pl;
+}
+
 bool decode_tc_supported(int D, int G) { return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8); }
 
 // p.chunks on entry: the partial slots the workspace holds per (batch, KV head)
@@ -513,10 +521,10 @@ cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t str
       !encode_4d_sw128(&p.tm_v, p.v_cache, p.D, p.Hkv, p.W, p.B) ||
       !encode_2d_sw128(&p.tm_q, p.q, p.D, static_cast<int64_t>(p.B) * p.Hq, kTcdN))
     return cudaErrorInvalidValue;
-  p.chunks = decode_tc_pieces(p.B, p.Hkv, p.n_valid, p_in.chunks, sms);
-  p.chunk_len = cdiv(cdiv(p.n_valid, p.chunks), kTcdKeys) * kTcdKeys;
-  const int64_t units = static_cast<int64_t>(p.B) * p.Hkv * p.chunks;
-  const int grid = static_cast<int>(std::min<int64_t>(units, sms));
+  const DecodeTcPlan pl = decode_tc_plan(p.B, p.Hkv, p.n_valid, p_in.chunks, sms);
+  p.chunks = pl.pieces;
+  p.chunk_len = pl.piece_len;
+  const int grid = pl.grid;
   const int64_t n16 = static_cast<int64_t>(p.B) * p.Hkv * p.D / 8;
   decode_append_kernel<<<static_cast<int>(std::min<int64_t>(1024, (n16 + 255) / 256)), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();

@@ -117,6 +117,12 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
 // runs the persistent kernel and the combine; p.chunks = partial slots available
 bool decode_tc_supported(int D, int G);
 int decode_tc_pieces(int B, int Hkv, int n_valid, int max_pieces, int sms);
+// the launch the tensor-core decode makes: pieces of the valid window per
+// (batch, KV head), slots per piece (whole 128-key tiles), persistent CTAs
+struct DecodeTcPlan {
+  int pieces, piece_len, grid;
+};
+DecodeTcPlan decode_tc_plan(int B, int Hkv, int n_valid, int max_pieces, int sms);
 cudaError_t launch_decode_tc(const DecodeParams& p, int sms, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t stream);
 // bf16 [B, N, H, D] as a 4-D map {D, H, N, B}, box 64 x 1 x 128 x 1, 128-byte swizzle

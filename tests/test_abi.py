@@ -114,3 +114,39 @@ def test_stream_geometry_sizes(swa):
     assert n2 - n >= 2 * 290 * 16 * 16 * 64 * 2
     bad = swa._make_cfg(1, 16, 64, 1004, 8, 64, 16, False, 2000, 300, __import__("torch").bfloat16, 16)
     assert swa._lib.swa_stream_bytes(C.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("B,Hkv,W,pos", [(64, 8, 4096, 200000), (8, 8, 1024, 5000), (1, 1, 640, 639),
+                                         (2, 16, 300, 1000), (4, 8, 1024, 500), (3, 8, 256, 700),
+                                         (2, 1, 130, 129), (1, 8, 4096, 10), (1, 1, 5000, 4998),
+                                         (200, 8, 4096, 10**6), (3, 2, 64, 200), (2, 2, 64, 10)])
+def test_decode_plan_covers_the_valid_window(swa, B, Hkv, W, pos):
+    pl = swa.swa_sched_decode(B, Hkv, W, pos)
+    n_valid = min(pos + 1, W)
+    assert pl["n_valid"] == n_valid
+    # pieces fit the workspace's partial slots and are whole 128-key tiles
+    assert 1 <= pl["pieces"] <= pl["slots"]
+    assert pl["piece_len"] % 128 == 0 and pl["piece_len"] > 0
+    # the pieces [k*len, min((k+1)*len, n_valid)) cover the valid slots exactly once
+    covered = []
+    for k in range(pl["pieces"]):
+        lo, hi = k * pl["piece_len"], min((k + 1) * pl["piece_len"], n_valid)
+        if hi > lo:
+            covered.append((lo, hi))
+    assert covered[0][0] == 0 and covered[-1][1] == n_valid
+    assert all(a[1] == b[0] for a, b in zip(covered, covered[1:]))
+    # one CTA per SM at most, none idle when units run short
+    assert pl["grid"] == min(B * Hkv * pl["pieces"], 148)
+    # the workspace the caller sizes holds every partial the plan writes
+    G = 4
+    need = swa.swa_decode_workspace_bytes(B, Hkv * G, Hkv, 128, W)
+    assert need >= B * Hkv * pl["pieces"] * G * (128 + 2) * 4
+
+
+def test_decode_plan_bench_shape_and_bad_args(swa):
+    # batch 64, 8 KV heads, 4096 slots: two halves per (batch, KV head), 1024 units on 148 CTAs
+    assert swa.swa_sched_decode(64, 8, 4096, 200000) == {"pieces": 2, "piece_len": 2048, "grid": 148,
+                                                          "slots": 8, "n_valid": 4096}
+    for bad in ((0, 8, 4096, 1), (1, 0, 4096, 1), (1, 8, 0, 1), (1, 8, 4096, -1)):
+        with pytest.raises(swa.SwaError):
+            swa.swa_sched_decode(*bad)
