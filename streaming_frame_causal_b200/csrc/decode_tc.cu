@@ -510,7 +510,9 @@ DecodeTcPlan decode_tc_plan(int B, int Hkv, int n_valid, int max_pieces, int sms
   return pl;
 }
 
-bool decode_tc_supported(int D, int G) { return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8); }
+bool decode_tc_supported(int D, int G) {
+  return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
+}
 
 // p.chunks on entry: the partial slots the workspace holds per (batch, KV head)
 cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t stream) {
