@@ -357,12 +357,14 @@ def run_ours(args, rank, world, local_rank):
     if "prefill" in per:
         parts_out["prefill_tflops"] = flops_prefill() / (per["prefill"] * 1e-3) / 1e12
         parts_out["prefill_ms"] = per["prefill"]
-        parts_out["prefill_frac_of_bf16"] = parts_out["prefill_tflops"] / peaks["bf16_tflops_sustained"]
+        parts_out["prefill_frac_of_bf16"] = parts_out["prefill_tflops"] / peaks["bf16_tflops"]
+        parts_out["prefill_frac_of_bf16_sustained"] = parts_out["prefill_tflops"] / peaks["bf16_tflops_sustained"]
     if "stream" in per:
         parts_out["stream_frames_per_s"] = ST["frames_per_step"] / (per["stream"] * 1e-3)
         parts_out["stream_ms_per_frame"] = per["stream"] / ST["frames_per_step"]
         parts_out["stream_tflops"] = stage_flops["stream"] / (per["stream"] * 1e-3) / 1e12
-        parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
+        parts_out["stream_frac_of_bf16"] = parts_out["stream_tflops"] / peaks["bf16_tflops"]
+        parts_out["stream_frac_of_bf16_sustained"] = parts_out["stream_tflops"] / peaks["bf16_tflops_sustained"]
         lat = sorted(fev[s][j].elapsed_time(fev[s][j + 1]) for s in range(args.steps)
                      for j in range(ST["frames_per_step"]))
         parts_out["stream_frame_ms_p50"] = lat[len(lat) // 2]
@@ -413,12 +415,15 @@ def run_ours(args, rank, world, local_rank):
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
         parts_out["band_ms"] = per["band"]
-        parts_out["band_frac_of_bf16"] = parts_out["band_tflops"] / peaks["bf16_tflops_sustained"]
+        parts_out["band_frac_of_bf16"] = parts_out["band_tflops"] / peaks["bf16_tflops"]
+        parts_out["band_frac_of_bf16_sustained"] = parts_out["band_tflops"] / peaks["bf16_tflops_sustained"]
     if "decode" in per:
         parts_out["decode_tok_per_s"] = DC["B"] / (per["decode"] * 1e-3)
         parts_out["decode_us"] = per["decode"] * 1e3
         parts_out["decode_gbs"] = decode_bytes() / (per["decode"] * 1e-3) / 1e9
         parts_out["decode_frac_of_hbm"] = parts_out["decode_gbs"] / peaks["hbm_gbs"]
+        # the decode target is stated against about 8 TB/s of HBM3e bandwidth
+        parts_out["decode_frac_of_8tbs"] = parts_out["decode_gbs"] / 8000.0
 
     # roofline of the dominant kernel: the kernel with the largest summed time in
     # the step.  attn_tc_kernel<64> runs the prefill launch and the eight
@@ -444,11 +449,14 @@ def run_ours(args, rank, world, local_rank):
     _, kms, kname, kwork, tkey, bound = max(cands)
     if bound == "tensor":
         achieved = kwork / (kms * 1e-3) / 1e12
+        # the dominant launch lasts about 2 ms at full clock inside a sub-second
+        # timed region: the burst bf16 figure is its peak; the sustained one (a
+        # seconds-long power-capped loop) is kept as a second reference
         roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"],
-                "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside the step); "
-                             f"frac of burst {achieved / peaks['bf16_tflops']:.3f}",
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_note": f"{peaks['source']} burst bf16 peak",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": recorded_traffic(tkey)}
     else:
         achieved = kwork / (kms * 1e-3) / 1e9

@@ -145,15 +145,25 @@ typedef struct swa_stream_cfg {
 
 typedef struct swa_stream swa_stream;  /* opaque host handle */
 
-/* Device bytes swa_stream_create needs for ``cfg`` (0 if cfg is invalid). */
-size_t swa_stream_bytes(const swa_stream_cfg* cfg);
+/* Device bytes swa_stream_init needs for ``cfg`` (0 if cfg is invalid): every
+ * layer's metadata and K/V pages plus the split-KV partials of the attend. */
+size_t swa_stream_cache_bytes(const swa_stream_cfg* cfg);
 
 /* Create a handle over ``dev_buf`` (caller-owned device memory of at least
- * swa_stream_bytes(cfg) bytes, 256-byte aligned).  Clears the buffer on ``stream``.
- * The handle is host memory owned by the library until swa_stream_destroy. */
+ * swa_stream_cache_bytes(cfg) bytes, 256-byte aligned).  Clears the buffer on
+ * ``stream`` and waits for it.  The handle is host memory owned by the library
+ * until swa_stream_destroy; the library allocates no device memory.  Errors:
+ * SWA_ERR_ARG (invalid cfg, null or misaligned buffer), SWA_ERR_CAPACITY (bytes
+ * too small), SWA_ERR_UNSUPPORTED (dtype / head_dim not built). */
+swa_status swa_stream_init(swa_stream** out, const swa_stream_cfg* cfg, void* dev_buf,
+                           size_t bytes, void* stream);
+void swa_stream_destroy(swa_stream* h);
+
+/* Earlier names of swa_stream_cache_bytes and swa_stream_init, kept as aliases
+ * (same arguments, same behaviour). */
+size_t swa_stream_bytes(const swa_stream_cfg* cfg);
 swa_status swa_stream_create(swa_stream** out, const swa_stream_cfg* cfg, void* dev_buf,
                              size_t bytes, void* stream);
-void swa_stream_destroy(swa_stream* h);
 
 /* Empty every layer's cache (the pages' clean_kv_cache). */
 swa_status swa_stream_reset(swa_stream* h, void* stream);
@@ -255,10 +265,41 @@ typedef struct swa_meta_layout {
 
 swa_status swa_stream_meta_layout(const swa_stream* h, swa_meta_layout* out);
 
-/* Synchronous copy of layer ``global_idx``'s metadata block into host ``dst``
- * (n_ints >= layout.n_ints).  For tests and inspection; waits for ``stream``. */
-swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, int32_t* dst,
-                               size_t n_ints, void* stream);
+/* Host view of one layer's cache bookkeeping ([AGG] "KV Cache Eviction
+ * Strategy": which frames the cache holds, where, and what the last append
+ * evicted).  The counts are always filled; each array is the caller's host
+ * memory, filled when non-NULL, and must hold its count (else
+ * SWA_ERR_CAPACITY). */
+typedef struct swa_meta_host {
+    int n_frames;          /* frames appended to the layer so far                    */
+    int n_evicted;         /* full frames evicted so far                             */
+    int n_special_tokens;  /* special tokens retained from evicted frames            */
+    int n_pages;           /* entries of the page table                              */
+    int n_segs;            /* key segments (contiguous storage runs) the attend reads */
+    int n_retained;        /* full frames the cache holds                            */
+    int n_slots;           /* slots of the layer (entries of slot_frame)             */
+    int n_last_evicted;    /* size of the last append's eviction set: 0 or 1         */
+    int last_evicted;      /* the frame it evicted, -1 if none                       */
+    int32_t* slot_frame;   /* [n_slots]: frame held by each slot, -1 empty           */
+    int slot_cap;
+    int32_t* page_table;   /* [n_pages]: physical page ids in logical key order      */
+    int page_cap;
+    int32_t* seg_row;      /* [n_segs]: first storage row of each key segment        */
+    int32_t* seg_len;      /* [n_segs]: tokens in each key segment                   */
+    int seg_cap;
+} swa_meta_host;
+
+/* Fill ``m`` with layer ``global_idx``'s bookkeeping: a synchronous copy from the
+ * device (waits for ``stream``), for tests and inspection.  Errors: SWA_ERR_ARG
+ * (null), SWA_ERR_CAPACITY (layer out of range, or an array too small),
+ * SWA_ERR_CUDA. */
+swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, swa_meta_host* m, void* stream);
+
+/* The same bookkeeping as the raw int32 block of swa_stream_meta_layout (header
+ * ints 0..7, then slot map, page table, segment rows and lengths) copied into
+ * host ``dst`` (n_ints >= layout.n_ints); synchronous. */
+swa_status swa_stream_get_meta_raw(const swa_stream* h, int global_idx, int32_t* dst,
+                                   size_t n_ints, void* stream);
 
 /* Device pointers of layer ``global_idx``'s K and V page storage
  * ([n_pages_total * page_tokens, heads, head_dim]); NULL on error. */
@@ -282,7 +323,10 @@ swa_status swa_band_prefill(const void* q, const void* k, const void* v, void* o
  *   k_cache, v_cache: [B, W, Hkv, head_dim] (updated in place).
  *   workspace: device scratch of at least swa_decode_workspace_bytes(...) bytes
  *   (split-K partials); calls sharing a workspace must not overlap on the GPU.
- * bf16: head_dim 64 or 128, Hq/Hkv <= 8; f32: 32, 64 or 128. */
+ * bf16: head_dim 64 or 128 with Hq/Hkv in {1, 2, 4, 8} (other group sizes return
+ * SWA_ERR_UNSUPPORTED); f32: head_dim 32, 64 or 128, any Hq/Hkv.  The kernels read
+ * only the valid slots' values: slots beyond ``pos`` may hold anything, NaN
+ * included. */
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int head_dim, int W);
 swa_status swa_decode(const void* q, const void* k_new, const void* v_new,
                       void* k_cache, void* v_cache, long long pos, int W,
@@ -323,9 +367,15 @@ swa_status swa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
 uint64_t swa_launch_count(void);
 
 /* ------------------------------------------------------- device errors
- * Kernels bound every wait; a wait that runs out latches a device flag and the
- * kernel returns early.  swa_device_error_check synchronizes ``stream``, reads and
- * clears the flag and returns SWA_ERR_TIMEOUT if it was set (SWA_OK otherwise).
+ * Kernels bound every wait; a wait that runs out latches a per-device flag and
+ * the kernel returns early.  The flag is mirrored into pinned, mapped host memory
+ * (a static page of the library, registered on first use), so once a kernel has
+ * latched an error every later call that would launch work on that device
+ * returns SWA_ERR_TIMEOUT at once, without synchronizing and without launching,
+ * until the error is cleared.  swa_device_error_check synchronizes ``stream``,
+ * reads and clears the flag and returns SWA_ERR_TIMEOUT if it was set (SWA_OK
+ * otherwise).  The first call on a device sets the flag up (a symbol lookup and
+ * a small synchronous copy): make it before any stream capture.
  * swa_debug_wait_timeout launches one thread that waits on a flag nothing sets for
  * ``timeout_us`` microseconds, so tests can exercise that path. */
 swa_status swa_device_error_check(void* stream);

@@ -45,6 +45,15 @@ class swa_stream_cfg(C.Structure):
         "cross_frame_special", "num_special", "max_frames", "dtype", "max_splits")]
 
 
+class swa_meta_host(C.Structure):
+    _fields_ = [(n, C.c_int) for n in (
+        "n_frames", "n_evicted", "n_special_tokens", "n_pages", "n_segs", "n_retained", "n_slots",
+        "n_last_evicted", "last_evicted")] + [
+        ("slot_frame", C.POINTER(C.c_int32)), ("slot_cap", C.c_int),
+        ("page_table", C.POINTER(C.c_int32)), ("page_cap", C.c_int),
+        ("seg_row", C.POINTER(C.c_int32)), ("seg_len", C.POINTER(C.c_int32)), ("seg_cap", C.c_int)]
+
+
 class swa_meta_layout(C.Structure):
     _fields_ = [(n, C.c_int) for n in (
         "n_ints", "n_slots", "pages_per_frame", "max_pages", "max_segs", "off_slot_frame",
@@ -59,6 +68,8 @@ _sigs = {
     "swa_sched_prefill": (_i64, [_i, _i, _i, _i, _i, _i, _i, _vp, _i64]),
     "swa_sched_decode": (_i, [_i, _i, _i, C.c_longlong, _i, _vp]),
     "swa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "swa_stream_cache_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
+    "swa_stream_init": (_i, [C.POINTER(_vp), C.POINTER(swa_stream_cfg), _vp, _sz, _vp]),
     "swa_stream_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
     "swa_stream_create": (_i, [C.POINTER(_vp), C.POINTER(swa_stream_cfg), _vp, _sz, _vp]),
     "swa_stream_destroy": (None, [_vp]),
@@ -70,7 +81,8 @@ _sigs = {
     "swa_stream_append_evict_pre": (_i, [_vp, _i, _i] + [_vp] * 10 + [C.c_float] + [_vp] * 3),
     "swa_rope3d_table": (_i, [_i, _i, _i, _i, _i, C.c_double, _vp, _vp]),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
-    "swa_stream_get_meta": (_i, [_vp, _i, _vp, _sz, _vp]),
+    "swa_stream_get_meta": (_i, [_vp, _i, C.POINTER(swa_meta_host), _vp]),
+    "swa_stream_get_meta_raw": (_i, [_vp, _i, _vp, _sz, _vp]),
     "swa_stream_k_storage": (_vp, [_vp, _i]),
     "swa_stream_v_storage": (_vp, [_vp, _i]),
     "swa_band_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
@@ -274,8 +286,11 @@ def _make_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_
                           SWA_BF16 if dtype == torch.bfloat16 else SWA_F32, max_splits)
 
 
-def swa_stream_bytes(**cfg) -> int:
-    return int(_lib.swa_stream_bytes(C.byref(_make_cfg(**cfg))))
+def swa_stream_cache_bytes(**cfg) -> int:
+    return int(_lib.swa_stream_cache_bytes(C.byref(_make_cfg(**cfg))))
+
+
+swa_stream_bytes = swa_stream_cache_bytes  # earlier name, same call
 
 
 class SwaStream:
@@ -287,13 +302,13 @@ class SwaStream:
                  device="cuda", stream=None):
         self.cfg = _make_cfg(num_layers, heads, head_dim, P, scale_frames, window_frames, page_tokens,
                              cross_frame_special, num_special, max_frames, dtype, max_splits)
-        self.nbytes = int(_lib.swa_stream_bytes(C.byref(self.cfg)))
+        self.nbytes = int(_lib.swa_stream_cache_bytes(C.byref(self.cfg)))
         if self.nbytes == 0:
-            raise SwaError(-1, "swa_stream_bytes")
+            raise SwaError(-1, "swa_stream_cache_bytes")
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
         h = C.c_void_p()
-        _check(_lib.swa_stream_create(C.byref(h), C.byref(self.cfg), self.buf.data_ptr(), self.nbytes,
-                                      _stream(stream)), "swa_stream_create")
+        _check(_lib.swa_stream_init(C.byref(h), C.byref(self.cfg), self.buf.data_ptr(), self.nbytes,
+                                    _stream(stream)), "swa_stream_init")
         self.handle = h
         lay = swa_meta_layout()
         _check(_lib.swa_stream_meta_layout(self.handle, C.byref(lay)), "swa_stream_meta_layout")
@@ -343,20 +358,35 @@ class SwaStream:
         return out
 
     def swa_stream_get_meta(self, global_idx: int, stream=None) -> dict:
+        """Layer ``global_idx``'s bookkeeping through the swa_meta_host view."""
         import numpy as np
         lay = self.layout
-        raw = np.zeros(lay.n_ints, dtype=np.int32)
-        _check(_lib.swa_stream_get_meta(self.handle, global_idx, raw.ctypes.data, lay.n_ints,
-                                        _stream(stream)), "swa_stream_get_meta")
-        n_pages, n_segs = int(raw[4]), int(raw[5])
+        slot = np.zeros(lay.n_slots, dtype=np.int32)
+        pages = np.zeros(lay.max_pages, dtype=np.int32)
+        srow = np.zeros(lay.max_segs, dtype=np.int32)
+        slen = np.zeros(lay.max_segs, dtype=np.int32)
+        ip = C.POINTER(C.c_int32)
+        m = swa_meta_host()
+        m.slot_frame, m.slot_cap = slot.ctypes.data_as(ip), lay.n_slots
+        m.page_table, m.page_cap = pages.ctypes.data_as(ip), lay.max_pages
+        m.seg_row, m.seg_len, m.seg_cap = srow.ctypes.data_as(ip), slen.ctypes.data_as(ip), lay.max_segs
+        _check(_lib.swa_stream_get_meta(self.handle, global_idx, C.byref(m), _stream(stream)),
+               "swa_stream_get_meta")
         return {
-            "n_frames": int(raw[0]), "n_evicted": int(raw[1]), "n_special": int(raw[2]),
-            "last_evicted": int(raw[3]), "n_pages": n_pages, "n_segs": n_segs, "n_retained": int(raw[6]),
-            "slot_frame": raw[lay.off_slot_frame:lay.off_slot_frame + lay.n_slots].copy(),
-            "page_table": raw[lay.off_page_table:lay.off_page_table + n_pages].copy(),
-            "seg_row": raw[lay.off_seg_row:lay.off_seg_row + n_segs].copy(),
-            "seg_len": raw[lay.off_seg_len:lay.off_seg_len + n_segs].copy(),
+            "n_frames": m.n_frames, "n_evicted": m.n_evicted, "n_special": m.n_special_tokens,
+            "last_evicted": m.last_evicted, "n_last_evicted": m.n_last_evicted, "n_pages": m.n_pages,
+            "n_segs": m.n_segs, "n_retained": m.n_retained, "slot_frame": slot[:m.n_slots].copy(),
+            "page_table": pages[:m.n_pages].copy(), "seg_row": srow[:m.n_segs].copy(),
+            "seg_len": slen[:m.n_segs].copy(),
         }
+
+    def swa_stream_get_meta_raw(self, global_idx: int, stream=None):
+        """Layer ``global_idx``'s raw int32 metadata block (layout: swa_stream_meta_layout)."""
+        import numpy as np
+        raw = np.zeros(self.layout.n_ints, dtype=np.int32)
+        _check(_lib.swa_stream_get_meta_raw(self.handle, global_idx, raw.ctypes.data, self.layout.n_ints,
+                                            _stream(stream)), "swa_stream_get_meta_raw")
+        return raw
 
     def storage(self, global_idx: int, which: str = "k") -> torch.Tensor:
         """View of a layer's K or V page storage as [rows, heads, head_dim]."""

@@ -29,10 +29,24 @@ void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std:
 extern "C" uint64_t swa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ device flag
+// The device error flag of each GPU is the first int of a 16-byte slot; its
+// second 8 bytes hold the device address of that GPU's word in a page of pinned,
+// mapped host memory (a static page of this library, registered once per
+// process: a registration, not an allocation).  Kernels that give up a bounded
+// wait set both (latch_error), so every entry point can refuse to launch while
+// an error is latched by reading host memory, with no device synchronization.
 namespace {
-__device__ int g_swa_err = 0;
+struct __align__(16) ErrSlot {
+  int flag;
+  int pad;
+  unsigned long long host;
+};
+__device__ ErrSlot g_swa_err = {0, 0, 0ull};
 
 constexpr int kMaxDevices = 64;
+constexpr int kHostWordStride = 16;  // ints: one 64-byte line per device
+alignas(4096) int g_host_err[kMaxDevices * kHostWordStride] = {0};
+bool g_host_err_mapped = false;
 int* g_err_ptr[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
 std::mutex g_mu;
@@ -43,16 +57,52 @@ int current_device() {
   return (d >= 0 && d < kMaxDevices) ? d : -1;
 }
 
+volatile int* host_err_word(int d) { return g_host_err + d * kHostWordStride; }
+
+// Device flag of the current device, set up on first use: its address, and the
+// host mirror word's device address written into the slot.  Without a mapped
+// host page (registration refused) the slot's host pointer stays 0 and latched
+// errors surface only through swa_device_error_check.
 int* err_ptr() {
   const int d = current_device();
   if (d < 0) return nullptr;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_err_ptr[d]) {
+    static bool tried = false;
+    if (!tried) {
+      tried = true;
+      g_host_err_mapped = cudaHostRegister(g_host_err, sizeof(g_host_err),
+                                           cudaHostRegisterMapped | cudaHostRegisterPortable) == cudaSuccess;
+      if (!g_host_err_mapped) cudaGetLastError();  // clear the error a refused registration leaves
+    }
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_swa_err) != cudaSuccess) return nullptr;
+    unsigned long long host_dev = 0;
+    if (g_host_err_mapped) {
+      void* hp = nullptr;
+      if (cudaHostGetDevicePointer(&hp, const_cast<int*>(host_err_word(d)), 0) == cudaSuccess)
+        host_dev = reinterpret_cast<unsigned long long>(hp);
+      else
+        cudaGetLastError();
+    }
+    if (cudaMemcpy(static_cast<uint8_t*>(p) + 8, &host_dev, sizeof(host_dev), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+      return nullptr;
     g_err_ptr[d] = static_cast<int*>(p);
   }
   return g_err_ptr[d];
+}
+
+// SWA_OK with *err = the current device's flag; SWA_ERR_TIMEOUT while an error
+// latched by an earlier launch on this device is uncleared; SWA_ERR_CUDA if the
+// flag cannot be set up.
+swa_status device_ready(int** err) {
+  int* e = err_ptr();
+  if (!e) return SWA_ERR_CUDA;
+  const int d = current_device();
+  if (d >= 0 && *host_err_word(d) != 0) return SWA_ERR_TIMEOUT;
+  *err = e;
+  return SWA_OK;
 }
 
 int num_sms() {
@@ -139,6 +189,7 @@ float scale_log2(int D) { return static_cast<float>(1.4426950408889634 / std::sq
 
 namespace swa {
 int* device_error_flag() { return err_ptr(); }
+int device_ready_status(int** err) { return device_ready(err); }
 }  // namespace swa
 
 // ==================================================================== status
@@ -221,8 +272,8 @@ extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, v
   if (B == 0 || S == 0) return SWA_OK;
   if (!q || !k || !v || !out) return SWA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_ARG;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int N = S * P;
   const int Wf = window_frames(sliding_window_size, num_frame_per_block);
@@ -282,8 +333,8 @@ extern "C" swa_status swa_band_prefill(const void* q, const void* k, const void*
   if (B == 0 || N == 0) return SWA_OK;
   if (!q || !k || !v || !out) return SWA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_ARG;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == SWA_F32) {
     if (!simt_head_dim(head_dim)) return SWA_ERR_UNSUPPORTED;
@@ -345,8 +396,8 @@ extern "C" swa_status swa_decode(const void* q, const void* k_new, const void* v
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
       !aligned16(v_cache) || !aligned16(out))
     return SWA_ERR_ARG;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DecodeParams p{};
   p.q = q;
@@ -474,14 +525,21 @@ uint8_t* layer_v(const swa_stream* h, int l) { return h->store0 + h->store_bytes
 
 }  // namespace
 
-extern "C" size_t swa_stream_bytes(const swa_stream_cfg* cfg) {
+extern "C" size_t swa_stream_cache_bytes(const swa_stream_cfg* cfg) {
   StreamGeom g;
   if (!stream_geom(cfg, &g)) return 0;
   return g.total;
 }
 
+extern "C" size_t swa_stream_bytes(const swa_stream_cfg* cfg) { return swa_stream_cache_bytes(cfg); }
+
 extern "C" swa_status swa_stream_create(swa_stream** out, const swa_stream_cfg* cfg, void* dev_buf,
                                         size_t bytes, void* stream) {
+  return swa_stream_init(out, cfg, dev_buf, bytes, stream);
+}
+
+extern "C" swa_status swa_stream_init(swa_stream** out, const swa_stream_cfg* cfg, void* dev_buf,
+                                      size_t bytes, void* stream) {
   if (!out || !cfg || !dev_buf) return SWA_ERR_ARG;
   *out = nullptr;
   StreamGeom g;
@@ -539,6 +597,8 @@ extern "C" void swa_stream_destroy(swa_stream* h) { delete h; }
 
 extern "C" swa_status swa_stream_reset(swa_stream* h, void* stream) {
   if (!h) return SWA_ERR_ARG;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // metadata: all -1 (empty slots, no eviction); counters rewritten per append
   cudaError_t e = cudaMemsetAsync(h->meta0, 0xff, h->meta_stride * h->cfg.num_layers, st);
@@ -594,8 +654,8 @@ extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int
   if (!k_frame || !v_frame || !aligned16(k_frame) || !aligned16(v_frame)) return SWA_ERR_ARG;
   if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
   if (frame_idx >= h->cfg.max_frames) return SWA_ERR_CAPACITY;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   const AppendParams p = append_params(h, global_idx, frame_idx, k_frame, v_frame, err);
   const cudaError_t e = launch_append_evict(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return SWA_ERR_CUDA;
@@ -615,8 +675,8 @@ swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, con
                         const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
                         const float* kn_b, const float* rot, int P, int C, int heads, float eps, void* xn_ws,
                         void* q_out, uint8_t* k_dst, uint8_t* v_dst, cudaStream_t st) {
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
   PreParams p;
   std::memset(&p, 0, sizeof(p));
@@ -663,6 +723,8 @@ extern "C" swa_status swa_rope3d_table(int frame_idx, int P, int num_special, in
     return SWA_ERR_ARG;
   if (P == 0) return SWA_OK;
   if (!rot_out || !aligned16(rot_out)) return SWA_ERR_ARG;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   return cuda_status(launch_rope3d_table(rot_out, frame_idx, P, num_special, grid_w, head_dim, theta,
                                          static_cast<cudaStream_t>(stream)));
 }
@@ -684,8 +746,8 @@ extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx,
     if (!q || !aligned16(q)) return SWA_ERR_ARG;
   if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
   if (frame_idx >= c.max_frames) return SWA_ERR_CAPACITY;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // eviction (the evicted frame's specials leave its slot first) and metadata,
   // then the prologue writes the frame's K/V into that slot
@@ -729,8 +791,8 @@ namespace {
 swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame, void* out, cudaStream_t st,
                               const int* hdr, const int* seg_row, const int* seg_len, int max_segs,
                               int n_frames_keys, int n_special) {
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   const swa_stream_cfg& c = h->cfg;
   if (c.dtype == SWA_F32) {
     SimtParams p{};
@@ -812,8 +874,8 @@ extern "C" swa_status swa_stream_attend_transient(swa_stream* h, int global_idx,
   if (!q_frame || !k_frame || !v_frame || !out || !aligned16(q_frame) || !aligned16(k_frame) ||
       !aligned16(v_frame) || !aligned16(out))
     return SWA_ERR_ARG;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const swa_stream_cfg& c = h->cfg;
   int* meta = layer_meta(h, global_idx);
@@ -858,8 +920,8 @@ extern "C" swa_status swa_stream_meta_layout(const swa_stream* h, swa_meta_layou
   return SWA_OK;
 }
 
-extern "C" swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, int32_t* dst, size_t n_ints,
-                                          void* stream) {
+extern "C" swa_status swa_stream_get_meta_raw(const swa_stream* h, int global_idx, int32_t* dst, size_t n_ints,
+                                              void* stream) {
   swa_status s = stream_check_layer(h, global_idx);
   if (s != SWA_OK) return s;
   if (!dst) return SWA_ERR_ARG;
@@ -869,6 +931,36 @@ extern "C" swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, i
                                   cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   return cuda_status(e);
+}
+
+extern "C" swa_status swa_stream_get_meta(const swa_stream* h, int global_idx, swa_meta_host* m, void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  if (!m) return SWA_ERR_ARG;
+  std::vector<int32_t> raw(static_cast<size_t>(h->meta_ints));
+  s = swa_stream_get_meta_raw(h, global_idx, raw.data(), raw.size(), stream);
+  if (s != SWA_OK) return s;
+  const int off_slot = 8, off_page = 8 + h->n_slots, off_row = off_page + h->max_pages,
+            off_len = off_row + h->max_segs;
+  m->n_frames = raw[0];
+  m->n_evicted = raw[1];
+  m->n_special_tokens = raw[2];
+  m->last_evicted = raw[3];
+  m->n_last_evicted = raw[3] >= 0 ? 1 : 0;
+  m->n_pages = raw[4];
+  m->n_segs = raw[5];
+  m->n_retained = raw[6];
+  m->n_slots = h->n_slots;
+  if (m->n_pages < 0 || m->n_pages > h->max_pages || m->n_segs < 0 || m->n_segs > h->max_segs)
+    return SWA_ERR_CUDA;  // the device metadata is not a state the append kernel writes
+  if ((m->slot_frame && m->slot_cap < m->n_slots) || (m->page_table && m->page_cap < m->n_pages) ||
+      ((m->seg_row || m->seg_len) && m->seg_cap < m->n_segs))
+    return SWA_ERR_CAPACITY;
+  if (m->slot_frame) std::memcpy(m->slot_frame, raw.data() + off_slot, sizeof(int32_t) * m->n_slots);
+  if (m->page_table) std::memcpy(m->page_table, raw.data() + off_page, sizeof(int32_t) * m->n_pages);
+  if (m->seg_row) std::memcpy(m->seg_row, raw.data() + off_row, sizeof(int32_t) * m->n_segs);
+  if (m->seg_len) std::memcpy(m->seg_len, raw.data() + off_len, sizeof(int32_t) * m->n_segs);
+  return SWA_OK;
 }
 
 extern "C" void* swa_stream_k_storage(const swa_stream* h, int global_idx) {
@@ -885,15 +977,19 @@ extern "C" void* swa_stream_v_storage(const swa_stream* h, int global_idx) {
 extern "C" swa_status swa_device_error_check(void* stream) {
   int* err = err_ptr();
   if (!err) return SWA_ERR_CUDA;
+  const int d = current_device();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, err, sizeof(int), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
+  // the stream is idle: the host mirror holds everything its kernels latched
+  if (d >= 0 && *host_err_word(d) != 0) v = 1;
   if (v != 0) {
     const int zero = 0;
     e = cudaMemcpyAsync(err, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (d >= 0) *host_err_word(d) = 0;
     return SWA_ERR_TIMEOUT;
   }
   return SWA_OK;
@@ -901,8 +997,8 @@ extern "C" swa_status swa_device_error_check(void* stream) {
 
 extern "C" swa_status swa_debug_wait_timeout(int timeout_us, void* stream) {
   if (timeout_us < 1 || timeout_us > 10000000) return SWA_ERR_ARG;
-  int* err = err_ptr();
-  if (!err) return SWA_ERR_CUDA;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   return cuda_status(launch_debug_wait(err, static_cast<long long>(timeout_us) * 1000, static_cast<cudaStream_t>(stream)));
 }
 
@@ -910,5 +1006,7 @@ extern "C" swa_status swa_debug_exp2_poly(const float* x, float* y, int n, void*
   if (n < 0) return SWA_ERR_ARG;
   if (n == 0) return SWA_OK;
   if (!x || !y) return SWA_ERR_ARG;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
   return cuda_status(launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
 }

@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
     glen = p.seg_len;
     nseg = p.meta_hdr[5];
     if (nseg < 0 || nseg > p.max_segs) {
-      if (lane == 0) atomicOr(p.err, ERR_BAD_META);
+      if (lane == 0) latch_error(p.err, ERR_BAD_META);
       return;
     }
   } else {  // SIMT_DECODE

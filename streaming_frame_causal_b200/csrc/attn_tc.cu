@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t ring = base + (is_k ? PL::kOffK : PL::kOffV);
       Cursor cur;
       bool ok = cursor_seek(w, w.t_begin, cur);
-      if (!ok) atomicOr(p.err, ERR_BAD_META);
+      if (!ok) latch_error(p.err, ERR_BAD_META);
       int issued = 0;
       for (int j = 0; j < T && ok; ++j) {
         const int st = j % PL::kStages;
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           break;
         }
         if (cur.s >= w.nseg) {
-          atomicOr(p.err, ERR_BAD_META);
+          latch_error(p.err, ERR_BAD_META);
           ok = false;
           break;
         }
@@ -714,11 +714,10 @@ int tc_smem_bytes(int head_dim) {
 namespace {
 template <int D>
 cudaError_t launch_tc_d(const TcParams& p, int64_t n_items, cudaStream_t stream) {
-  static int attr_dev_mask = 0;  // devices on which the smem opt-in was set (first 31)
+  static DeviceOnce attr_set;  // devices on which the smem opt-in was set
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  const int bit = 1 << (dev & 31);
-  if (!(attr_dev_mask & bit)) {
+  if (!attr_set.done(dev)) {
     // the setmaxnreg split moves registers inside the pool the CTA is launched
     // with; refuse to launch a build whose pool would be too small (the
     // increasing warpgroups would otherwise wait forever)
@@ -728,7 +727,7 @@ cudaError_t launch_tc_d(const TcParams& p, int64_t n_items, cudaStream_t stream)
     if (fa.numRegs * 12 < 4 * kRegsCtl + 8 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_dev_mask |= bit;
+    attr_set.mark(dev);
   }
   attn_tc_kernel<D><<<static_cast<unsigned>(n_items), kThreads, Plan<D>::kSmemBytes, stream>>>(p);
   count_launches(1);

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
   const int n_pages = n_ret * p.ppf + sp_pages;
   const int n_segs = n_ret + (n_special > 0 ? 1 : 0);
   if (n_pages > p.max_pages || n_segs > p.max_segs) {
-    if (threadIdx.x == 0) atomicOr(p.err, ERR_BAD_META);
+    if (threadIdx.x == 0) latch_error(p.err, ERR_BAD_META);
     return;
   }
   // retained frame with ordinal o (ascending frame index)
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(256) transient_prepare_kernel(const TransientP
   int* tlen = trow + (p.max_segs + 1);
   int n = hdr[5];
   if (n < 0 || n > p.max_segs) {
-    if (threadIdx.x == 0) atomicOr(p.err, ERR_BAD_META);
+    if (threadIdx.x == 0) latch_error(p.err, ERR_BAD_META);
     n = 0;
   }
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
@@ -166,7 +166,7 @@ __global__ void debug_wait_kernel(int* err, long long timeout_ns) {
   const uint64_t t0 = global_timer_ns();
   while (*reinterpret_cast<volatile int*>(&flag) == 0) {
     if (global_timer_ns() - t0 > static_cast<uint64_t>(timeout_ns)) {
-      atomicOr(err, ERR_WAIT_DEBUG);
+      latch_error(err, ERR_WAIT_DEBUG);
       return;
     }
   }

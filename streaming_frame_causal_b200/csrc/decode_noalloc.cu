@@ -74,9 +74,10 @@ extern "C" swa_status swa_decode_noalloc(const void* q, const void* k_new, const
   if (!q || !k_new || !v_new || !k_cache || !v_cache || !out) return SWA_ERR_ARG;
   if (!al16(q) || !al16(k_new) || !al16(v_new) || !al16(k_cache) || !al16(v_cache) || !al16(out))
     return SWA_ERR_ARG;
+  int* err = nullptr;
+  if (const int ds = swa::device_ready_status(&err)) return static_cast<swa_status>(ds);
   void* scratch = scratch_on_current_device();
-  int* err = swa::device_error_flag();
-  if (!scratch || !err) return SWA_ERR_CUDA;
+  if (!scratch) return SWA_ERR_CUDA;
 
   swa::DecodeParams p{};
   p.q = q;

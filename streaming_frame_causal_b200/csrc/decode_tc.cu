@@ -87,6 +87,10 @@ SWA_DEV void st_shared_b16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
+SWA_DEV void st_shared_zero16(uint32_t addr) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+}
+
 struct TcdUnit {
   int b, kvh, piece, t_begin, t_end, T;
 };
@@ -326,6 +330,17 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
         tmem_ld16(tmem + lane_off + sb * kTcdN, sv);
         tmem_wait_ld();
         const bool valid = u.t_begin + j * kTcdKeys + r < u.t_end;
+        if (!valid) {
+          // A key past the valid window still has a V row in the tile: cache
+          // slots the caller never wrote.  Its P is 0, but 0 x NaN is NaN, so
+          // the row is zeroed before the second product reads it (the
+          // proxy fence before the p_full arrival orders these stores first).
+          const uint32_t vrow = base + (jj % kTcdStages) * kTcdStage + kTcdTile + r * 128;
+#pragma unroll
+          for (int sub = 0; sub < PL::kSubs; ++sub)
+#pragma unroll
+            for (int c = 0; c < 128; c += 16) st_shared_zero16(vrow + sub * kTcdSub + c);
+        }
         float x[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) x[h] = valid ? __uint_as_float(sv[h]) * sl2 : -INFINITY;
@@ -465,15 +480,14 @@ __global__ void decode_append_kernel(const DecodeParams p) {
 template <int D, int G>
 cudaError_t launch_tcd(const DecodeParams& p, int grid, cudaStream_t stream) {
   constexpr int kSmem = TcdPlan<D>::kSmem;
-  static int attr_dev_mask = 0;
+  static DeviceOnce attr_set;  // devices on which the smem opt-in was set
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  const int bit = 1 << (dev & 31);
-  if (!(attr_dev_mask & bit)) {
+  if (!attr_set.done(dev)) {
     const cudaError_t e =
         cudaFuncSetAttribute(decode_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    attr_dev_mask |= bit;
+    attr_set.mark(dev);
   }
   decode_tc_kernel<D, G><<<grid, kTcdThreads, kSmem, stream>>>(p);
   return cudaGetLastError();

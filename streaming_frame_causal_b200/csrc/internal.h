@@ -3,9 +3,24 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace swa {
+
+// One bit per device (ids 0..63) recording that a per-device setting, such as a
+// kernel's shared-memory opt-in, has been made; safe for concurrent host
+// threads.  Devices beyond 63 are never marked, so the setting is simply
+// repeated on every call there.
+struct DeviceOnce {
+  std::atomic<uint64_t> mask{0};
+  bool done(int dev) const {
+    return dev >= 0 && dev < 64 && ((mask.load(std::memory_order_acquire) >> dev) & 1u);
+  }
+  void mark(int dev) {
+    if (dev >= 0 && dev < 64) mask.fetch_or(uint64_t{1} << dev, std::memory_order_acq_rel);
+  }
+};
 
 enum TcMode : int { TC_FRAME = 0, TC_STREAM = 1, TC_BAND = 2 };
 
@@ -162,6 +177,9 @@ cudaError_t launch_decode_write_f32(const DecodeParams& p, cudaStream_t stream);
 // ---------------------------------------------------------------- misc
 // device address of the library's error flag on the current device (nullptr on failure)
 int* device_error_flag();
+// 0 (SWA_OK) with *err = that flag; SWA_ERR_TIMEOUT while an error latched by an
+// earlier launch on the device is uncleared; SWA_ERR_CUDA if the flag cannot be set up
+int device_ready_status(int** err);
 // counts kernel launches (every launch_* helper adds what it enqueued)
 void count_launches(int n);
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);

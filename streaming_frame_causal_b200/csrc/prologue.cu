@@ -332,15 +332,14 @@ __global__ void rope3d_table_kernel(float* __restrict__ rot, int frame, int P, i
 
 template <int D>
 cudaError_t launch_pre_d(const PreParams& p, cudaStream_t stream) {
-  static int attr_dev_mask = 0;
+  static DeviceOnce attr_set;  // devices on which the smem opt-in was set
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  const int bit = 1 << (dev & 31);
-  if (!(attr_dev_mask & bit)) {
+  if (!attr_set.done(dev)) {
     const cudaError_t e =
         cudaFuncSetAttribute(qkv_pre_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmem);
     if (e != cudaSuccess) return e;
-    attr_dev_mask |= bit;
+    attr_set.mark(dev);
   }
   dim3 grid(cdiv(p.P, kPreM), 3 * p.C / kPreN);
   qkv_pre_kernel<D><<<grid, kPreThreads, kPreSmem, stream>>>(p);

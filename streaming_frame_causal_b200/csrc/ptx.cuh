@@ -64,6 +64,20 @@ SWA_DEV bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// The library's device error flag is the first int of a 16-byte slot whose
+// second 8 bytes hold a device-visible pointer to a word of pinned, mapped host
+// memory (or 0).  latch_error sets ``code`` in the device flag and mirrors it
+// into that host word, so the host sees a latched error on its next call
+// without synchronizing.
+SWA_DEV void latch_error(int* err, int code) {
+  atomicOr(err, code);
+  int* host = reinterpret_cast<int*>(*reinterpret_cast<volatile unsigned long long*>(err + 2));
+  if (host) {
+    __threadfence_system();
+    *reinterpret_cast<volatile int*>(host) = code;
+  }
+}
+
 // Wait for the phase with the given parity to complete.  Gives up when the
 // deadline passes or when another thread has already latched an error; on
 // giving up it latches ``code`` and returns false.
@@ -75,7 +89,7 @@ SWA_DEV bool mbar_wait(uint32_t addr, uint32_t parity, int* err, int code) {
     if ((it & 31u) == 0) {
       if (*reinterpret_cast<volatile int*>(err) != 0) return false;
       if (global_timer_ns() - t0 > SWA_WAIT_NS) {
-        atomicOr(err, code);
+        latch_error(err, code);
         return false;
       }
     }

@@ -25,6 +25,44 @@ def test_every_header_function_is_exported(swa):
     assert not missing, missing
 
 
+# the C ABI the hot path's scope names (prefill, stream cache, decode), by name
+SECTION_B_NAMES = ("swa_prefill", "swa_stream_cache_bytes", "swa_stream_init", "swa_stream_reset",
+                   "swa_stream_append_evict", "swa_stream_attend", "swa_stream_get_meta", "swa_decode",
+                   "swa_status_str")
+
+
+def test_boundary_names_are_exported(swa):
+    lib = C.CDLL(swa.LIB_PATH)
+    assert all(hasattr(lib, n) for n in SECTION_B_NAMES)
+    declared = set(swa.header_functions())
+    assert set(SECTION_B_NAMES) <= declared
+    # the earlier names stay as aliases of the same calls
+    assert {"swa_stream_bytes", "swa_stream_create", "swa_stream_get_meta_raw"} <= declared
+
+
+def test_meta_host_struct_matches_header(swa):
+    # field order and types of swa_meta_host as include/swa.h declares them
+    with open(swa.HEADER_PATH) as f:
+        text = f.read()
+    body = text[text.index("typedef struct swa_meta_host {"):text.index("} swa_meta_host;")]
+    import re
+    fields = re.findall(r"^\s*(int32_t\*|int)\s+(\w+);", body, re.M)
+    assert [n for _, n in fields] == [n for n, _ in swa.swa_meta_host._fields_]
+    for (ctype, name), (_, ftype) in zip(fields, swa.swa_meta_host._fields_):
+        assert (ctype == "int") == (ftype is C.c_int), name
+
+
+def test_meta_and_cache_bytes_reject_bad_args(swa):
+    lib = swa._lib
+    m = swa.swa_meta_host()
+    assert lib.swa_stream_get_meta(None, 0, C.byref(m), None) == -1
+    assert lib.swa_stream_get_meta_raw(None, 0, None, 0, None) == -1
+    cfg = swa._make_cfg(1, 16, 64, 1004, 8, 64, 16, False, 5, 300, __import__("torch").bfloat16, 12)
+    assert lib.swa_stream_cache_bytes(C.byref(cfg)) == lib.swa_stream_bytes(C.byref(cfg)) > 0
+    h = C.c_void_p()
+    assert lib.swa_stream_init(C.byref(h), C.byref(cfg), None, 0, None) == -1
+
+
 def test_status_strings(swa):
     assert swa.swa_status_str(0) == "ok"
     assert swa.swa_status_str(-3) == "frame out of order"
