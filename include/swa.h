@@ -113,6 +113,20 @@ swa_status swa_prefill(const void* q, const void* k, const void* v, void* out,
                        int sliding_window_size, int num_frame_per_block,
                        int num_frame_for_scale, int dtype, void* stream);
 
+/* Head-sliced prefill: the same attention on heads [head0, head0 + heads) of
+ * token rows ``row_stride`` elements apart, read and written in place.  q, k, v
+ * and out all point at the start of the full tensors [B, S*P, row_stride]; only
+ * the slice's elements are read or written.  This is how one GPU of several
+ * takes its share of the heads (each head is independent; no exchange inside the
+ * attention): rank r attends its heads of the same [B, S*P, C] tensors and an
+ * all-gather of the slices rebuilds the output.  Needs row_stride >= (head0 +
+ * heads) * head_dim (else SWA_ERR_SHAPE) and row_stride * element size a
+ * multiple of 16 bytes (else SWA_ERR_ARG); otherwise as swa_prefill. */
+swa_status swa_prefill_heads(const void* q, const void* k, const void* v, void* out,
+                             int B, int S, int P, int row_stride, int head0, int heads, int head_dim,
+                             int sliding_window_size, int num_frame_per_block,
+                             int num_frame_for_scale, int dtype, void* stream);
+
 /* --------------------------------------------------------- streaming cache
  * Per-layer rolling paged KV cache for frame-by-frame streaming ([AGG] "KV Cache
  * Eviction Strategy"; [BLK]).  ``global_idx`` selects the layer's cache.
@@ -186,6 +200,19 @@ swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx,
 swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx,
                              const void* q_frame, void* out, void* stream);
 
+/* Head-sliced forms of the append and the attend: the cache holds cfg.heads
+ * heads, taken from heads [head0, head0 + cfg.heads) of frame tensors whose token
+ * rows are ``row_stride`` elements apart (k_frame, v_frame, q_frame and out point
+ * at the full [P, row_stride] frames; the attend writes only its heads of out).
+ * One GPU of several keeps the cache of its share of the heads this way; the
+ * result equals the unsliced call on those heads.  Needs row_stride >= (head0 +
+ * cfg.heads) * head_dim (else SWA_ERR_SHAPE) and row_stride * element size a
+ * multiple of 16 bytes (else SWA_ERR_ARG); otherwise as the unsliced calls. */
+swa_status swa_stream_append_evict_heads(swa_stream* h, int global_idx, int frame_idx, const void* k_frame,
+                                         const void* v_frame, int row_stride, int head0, void* stream);
+swa_status swa_stream_attend_heads(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
+                                   void* out, int row_stride, int head0, void* stream);
+
 /* Non-keyframe attend ("Non-keyframe path" of the streaming attention block,
  * lingbot-map AggregatorStream guide: append with eviction deferred, attend,
  * roll the append back).  The queries q_frame [P, heads, head_dim] attend to
@@ -247,6 +274,29 @@ swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_
  * small head_dim, theta <= 1, null or misaligned output). */
 swa_status swa_rope3d_table(int frame_idx, int P, int num_special, int grid_w, int head_dim, double theta,
                             float* rot_out, void* stream);
+
+/* swa_attn_pre with the 3-D RoPE generated inside the prologue instead of read
+ * from a table (the I/O page's enable_3d_rope: positions built internally).  The
+ * positions and bands are those of swa_rope3d_table for (frame_idx, num_special,
+ * grid_w, theta); the epilogue forms each pair's angle pos * theta^(-j/n), reduces
+ * it to [-pi, pi] in double and takes its sine and cosine in float, so no table
+ * goes through device memory.  Other arguments, layouts and errors as
+ * swa_attn_pre, plus SWA_ERR_ARG for a negative frame_idx, num_special outside
+ * [0, P], grid_w < 1 or theta <= 1. */
+swa_status swa_attn_pre_rope3d(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
+                               const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
+                               const float* kn_b, int frame_idx, int num_special, int grid_w, double theta,
+                               int P, int C, int heads, float eps, void* xn_ws, void* q_out, void* k_out,
+                               void* v_out, void* stream);
+
+/* swa_stream_append_evict_pre with the 3-D RoPE of frame ``frame_idx`` generated
+ * inside the prologue (as swa_attn_pre_rope3d; num_special here is the RoPE's
+ * count of special tokens at (t, 0, 0), independent of the cache's retention). */
+swa_status swa_stream_append_evict_pre_rope3d(swa_stream* h, int global_idx, int frame_idx, const void* x,
+                                              const float* ln_w, const float* ln_b, const void* w_qkv,
+                                              const float* b_qkv, const float* qn_w, const float* qn_b,
+                                              const float* kn_w, const float* kn_b, int num_special, int grid_w,
+                                              double theta, float eps, void* xn_ws, void* q_out, void* stream);
 
 /* Layout of one layer's metadata block, in int32 units. */
 typedef struct swa_meta_layout {

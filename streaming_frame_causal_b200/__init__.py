@@ -68,6 +68,9 @@ _sigs = {
     "swa_sched_prefill": (_i64, [_i, _i, _i, _i, _i, _i, _i, _vp, _i64]),
     "swa_sched_decode": (_i, [_i, _i, _i, C.c_longlong, _i, _vp]),
     "swa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "swa_prefill_heads": (_i, [_vp, _vp, _vp, _vp] + [_i] * 11 + [_vp]),
+    "swa_stream_append_evict_heads": (_i, [_vp, _i, _i, _vp, _vp, _i, _i, _vp]),
+    "swa_stream_attend_heads": (_i, [_vp, _i, _i, _vp, _vp, _i, _i, _vp]),
     "swa_stream_cache_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
     "swa_stream_init": (_i, [C.POINTER(_vp), C.POINTER(swa_stream_cfg), _vp, _sz, _vp]),
     "swa_stream_bytes": (_sz, [C.POINTER(swa_stream_cfg)]),
@@ -80,6 +83,9 @@ _sigs = {
     "swa_attn_pre": (_i, [_vp] * 10 + [_i, _i, _i, C.c_float] + [_vp] * 5),
     "swa_stream_append_evict_pre": (_i, [_vp, _i, _i] + [_vp] * 10 + [C.c_float] + [_vp] * 3),
     "swa_rope3d_table": (_i, [_i, _i, _i, _i, _i, C.c_double, _vp, _vp]),
+    "swa_attn_pre_rope3d": (_i, [_vp] * 9 + [_i, _i, _i, C.c_double, _i, _i, _i, C.c_float] + [_vp] * 5),
+    "swa_stream_append_evict_pre_rope3d": (_i, [_vp, _i, _i] + [_vp] * 9 + [_i, _i, C.c_double, C.c_float]
+                                           + [_vp] * 3),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
     "swa_stream_get_meta": (_i, [_vp, _i, C.POINTER(swa_meta_host), _vp]),
     "swa_stream_get_meta_raw": (_i, [_vp, _i, _vp, _sz, _vp]),
@@ -184,6 +190,26 @@ def swa_prefill(q, k, v, out, S: int, P: int, sliding_window_size: int, num_fram
     return out
 
 
+def head_shard(rank: int, world: int, heads: int) -> tuple[int, int]:
+    """(head0, count) of rank ``rank``'s share when ``world`` GPUs split ``heads``
+    attention heads (contiguous, as even as possible, lower ranks taking the
+    extra head)."""
+    if world < 1 or not 0 <= rank < world or heads < world:
+        raise ValueError("need 0 <= rank < world <= heads")
+    base, extra = divmod(heads, world)
+    return rank * base + min(rank, extra), base + (1 if rank < extra else 0)
+
+
+def swa_prefill_heads(q, k, v, out, S: int, P: int, head0: int, heads: int, sliding_window_size: int,
+                      num_frame_per_block: int = 1, num_frame_for_scale: int = 0, stream=None) -> torch.Tensor:
+    """swa_prefill on heads [head0, head0 + heads) of q/k/v/out [B, S*P, H, D], in place."""
+    B, N, H, D = q.shape
+    _check(_lib.swa_prefill_heads(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, P, H * D, head0, heads, D,
+                                  sliding_window_size, num_frame_per_block, num_frame_for_scale,
+                                  _dtype_code(q), _stream(stream)), "swa_prefill_heads")
+    return out
+
+
 def swa_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads: int, eps: float = 1e-6,
                  q_out=None, k_out=None, v_out=None, xn_ws=None, stream=None):
     """Attention prologue of one frame: x [P, C] bf16 -> q, k, v [P, heads, C/heads]
@@ -198,6 +224,25 @@ def swa_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, heads
     _check(_lib.swa_attn_pre(_ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv), _ptr(qn_w), _ptr(qn_b),
                              _ptr(kn_w), _ptr(kn_b), _ptr(rot), P, Cdim, heads, float(eps), _ptr(xn_ws),
                              _ptr(q_out), _ptr(k_out), _ptr(v_out), _stream(stream)), "swa_attn_pre")
+    return q_out, k_out, v_out
+
+
+def swa_attn_pre_rope3d(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, heads: int, frame_idx: int,
+                        num_special: int, grid_w: int, theta: float = 10000.0, eps: float = 1e-6, q_out=None,
+                        k_out=None, v_out=None, xn_ws=None, stream=None):
+    """swa_attn_pre with the frame's 3-D RoPE generated inside the prologue (no
+    table; positions and bands as swa_rope3d_table, see include/swa.h)."""
+    P, Cdim = x.shape
+    D = Cdim // heads
+    q_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if q_out is None else q_out
+    k_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if k_out is None else k_out
+    v_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if v_out is None else v_out
+    xn_ws = torch.empty_like(x) if xn_ws is None else xn_ws
+    _check(_lib.swa_attn_pre_rope3d(_ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv), _ptr(qn_w),
+                                    _ptr(qn_b), _ptr(kn_w), _ptr(kn_b), int(frame_idx), int(num_special),
+                                    int(grid_w), float(theta), P, Cdim, heads, float(eps), _ptr(xn_ws),
+                                    _ptr(q_out), _ptr(k_out), _ptr(v_out), _stream(stream)),
+           "swa_attn_pre_rope3d")
     return q_out, k_out, v_out
 
 
@@ -332,6 +377,20 @@ class SwaStream:
         _check(_lib.swa_stream_append_evict(self.handle, global_idx, frame_idx, _ptr(k_frame),
                                             _ptr(v_frame), _stream(stream)), "swa_stream_append_evict")
 
+    def swa_stream_append_evict_heads(self, global_idx: int, frame_idx: int, k_frame, v_frame, head0: int,
+                                      stream=None):
+        """Append heads [head0, head0 + cfg.heads) of k_frame / v_frame [P, H, D]."""
+        P, H, D = k_frame.shape
+        _check(_lib.swa_stream_append_evict_heads(self.handle, global_idx, frame_idx, _ptr(k_frame), _ptr(v_frame),
+                                                  H * D, head0, _stream(stream)), "swa_stream_append_evict_heads")
+
+    def swa_stream_attend_heads(self, global_idx: int, frame_idx: int, q_frame, out, head0: int, stream=None):
+        """Attend heads [head0, head0 + cfg.heads) of q_frame [P, H, D] into the same heads of out."""
+        P, H, D = q_frame.shape
+        _check(_lib.swa_stream_attend_heads(self.handle, global_idx, frame_idx, _ptr(q_frame), _ptr(out), H * D,
+                                            head0, _stream(stream)), "swa_stream_attend_heads")
+        return out
+
     def swa_stream_attend(self, global_idx: int, frame_idx: int, q_frame, out, stream=None):
         _check(_lib.swa_stream_attend(self.handle, global_idx, frame_idx, _ptr(q_frame), _ptr(out),
                                       _stream(stream)), "swa_stream_attend")
@@ -347,6 +406,18 @@ class SwaStream:
                                                 _ptr(w_qkv), _ptr(b_qkv), _ptr(qn_w), _ptr(qn_b), _ptr(kn_w),
                                                 _ptr(kn_b), _ptr(rot), float(eps), _ptr(xn_ws), _ptr(q_out),
                                                 _stream(stream)), "swa_stream_append_evict_pre")
+        return q_out
+
+    def swa_stream_append_evict_pre_rope3d(self, global_idx: int, frame_idx: int, x, ln_w, ln_b, w_qkv, b_qkv,
+                                           qn_w, qn_b, kn_w, kn_b, q_out, num_special: int, grid_w: int,
+                                           theta: float = 10000.0, eps: float = 1e-6, xn_ws=None, stream=None):
+        """swa_stream_append_evict_pre with the frame's 3-D RoPE generated inside
+        the prologue (see include/swa.h)."""
+        xn_ws = torch.empty_like(x) if xn_ws is None else xn_ws
+        _check(_lib.swa_stream_append_evict_pre_rope3d(
+            self.handle, global_idx, frame_idx, _ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv),
+            _ptr(qn_w), _ptr(qn_b), _ptr(kn_w), _ptr(kn_b), int(num_special), int(grid_w), float(theta),
+            float(eps), _ptr(xn_ws), _ptr(q_out), _stream(stream)), "swa_stream_append_evict_pre_rope3d")
         return q_out
 
     def swa_stream_attend_transient(self, global_idx: int, q_frame, k_frame, v_frame, out, stream=None):

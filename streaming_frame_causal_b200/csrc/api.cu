@@ -139,13 +139,16 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor [B, N, H, D] (D contiguous) as a 4-D map {D, H, N, B}; box = 64
 // columns x 1 head x 128 rows, 128-byte swizzle (one box = one 16 KB operand
 // sub-tile in the layout the tcgen05 descriptors expect).
-bool make_map(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B) {
+// row_elems: elements between consecutive tokens (0: H * D, a contiguous tensor;
+// larger when the map covers a head slice of wider token rows).
+bool make_map(CUtensorMap* m, const void* base, int D, int H, int64_t N, int B, int64_t row_elems = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  if (row_elems == 0) row_elems = static_cast<int64_t>(H) * D;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                                 static_cast<cuuint64_t>(N) * H * D * 2};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(row_elems) * 2,
+                                 static_cast<cuuint64_t>(N) * row_elems * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
@@ -262,16 +265,18 @@ extern "C" int swa_sched_decode(int B, int Hkv, int W, long long pos, int sms, i
 }
 
 // ==================================================================== prefill
-extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, void* out, int B, int S, int P,
-                                  int C, int heads, int head_dim, int sliding_window_size,
-                                  int num_frame_per_block, int num_frame_for_scale, int dtype, void* stream) {
-  if (B < 0 || S < 0 || P < 1 || heads < 1 || head_dim < 1 || num_frame_per_block < 1) return SWA_ERR_ARG;
-  if (dtype != SWA_F32 && dtype != SWA_BF16) return SWA_ERR_ARG;
-  if (C != heads * head_dim) return SWA_ERR_SHAPE;
-  if (static_cast<int64_t>(S) * P > 0x7fffffffLL) return SWA_ERR_SHAPE;
+namespace {
+// The prefill over heads [head0, head0 + heads) of token rows ``row_stride``
+// elements apart (the whole tensor when head0 = 0 and row_stride = heads * D).
+swa_status prefill_impl(const void* q, const void* k, const void* v, void* out, int B, int S, int P,
+                        int64_t row_stride, int head0, int heads, int head_dim, int sliding_window_size,
+                        int num_frame_per_block, int num_frame_for_scale, int dtype, void* stream) {
   if (B == 0 || S == 0) return SWA_OK;
   if (!q || !k || !v || !out) return SWA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_ARG;
+  const int esize = dtype == SWA_F32 ? 4 : 2;
+  if ((row_stride * esize) % 16 != 0 || (static_cast<int64_t>(head0) * head_dim * esize) % 16 != 0)
+    return SWA_ERR_ARG;
   int* err = nullptr;
   if (const swa_status ds = device_ready(&err)) return ds;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -297,15 +302,21 @@ extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, v
     p.S = Sc;
     p.Wf = Wf;
     p.scale = 1.f / std::sqrt(static_cast<float>(head_dim));
+    p.q_ld = p.kv_ld = row_stride;
+    p.q_h0 = p.kv_h0 = head0;
     return cuda_status(launch_attn_simt(p, st));
   }
   if (!tc_head_dim(head_dim)) return SWA_ERR_UNSUPPORTED;
+  const size_t off = static_cast<size_t>(head0) * head_dim * 2;
   TcParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tm_q, q, head_dim, heads, N, B) || !make_map(&p.tm_k, k, head_dim, heads, N, B) ||
-      !make_map(&p.tm_v, v, head_dim, heads, N, B))
+  if (!make_map(&p.tm_q, static_cast<const uint8_t*>(q) + off, head_dim, heads, N, B, row_stride) ||
+      !make_map(&p.tm_k, static_cast<const uint8_t*>(k) + off, head_dim, heads, N, B, row_stride) ||
+      !make_map(&p.tm_v, static_cast<const uint8_t*>(v) + off, head_dim, heads, N, B, row_stride))
     return SWA_ERR_CUDA;
   p.out = out;
+  p.out_ld = row_stride;
+  p.out_h0 = head0;
   p.err = err;
   p.mode = TC_FRAME;
   p.B = B;
@@ -322,6 +333,31 @@ extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, v
   const int64_t items = static_cast<int64_t>(S) * B * heads * p.n_pairs;
   if (items > 0x7fffffffLL) return SWA_ERR_SHAPE;
   return cuda_status(launch_attn_tc(p, head_dim, items, st));
+}
+}  // namespace
+
+extern "C" swa_status swa_prefill(const void* q, const void* k, const void* v, void* out, int B, int S, int P,
+                                  int C, int heads, int head_dim, int sliding_window_size,
+                                  int num_frame_per_block, int num_frame_for_scale, int dtype, void* stream) {
+  if (B < 0 || S < 0 || P < 1 || heads < 1 || head_dim < 1 || num_frame_per_block < 1) return SWA_ERR_ARG;
+  if (dtype != SWA_F32 && dtype != SWA_BF16) return SWA_ERR_ARG;
+  if (C != heads * head_dim) return SWA_ERR_SHAPE;
+  if (static_cast<int64_t>(S) * P > 0x7fffffffLL) return SWA_ERR_SHAPE;
+  return prefill_impl(q, k, v, out, B, S, P, C, 0, heads, head_dim, sliding_window_size, num_frame_per_block,
+                      num_frame_for_scale, dtype, stream);
+}
+
+extern "C" swa_status swa_prefill_heads(const void* q, const void* k, const void* v, void* out, int B, int S,
+                                        int P, int row_stride, int head0, int heads, int head_dim,
+                                        int sliding_window_size, int num_frame_per_block, int num_frame_for_scale,
+                                        int dtype, void* stream) {
+  if (B < 0 || S < 0 || P < 1 || heads < 1 || head_dim < 1 || num_frame_per_block < 1 || head0 < 0)
+    return SWA_ERR_ARG;
+  if (dtype != SWA_F32 && dtype != SWA_BF16) return SWA_ERR_ARG;
+  if (static_cast<int64_t>(row_stride) < static_cast<int64_t>(head0 + heads) * head_dim) return SWA_ERR_SHAPE;
+  if (static_cast<int64_t>(S) * P > 0x7fffffffLL) return SWA_ERR_SHAPE;
+  return prefill_impl(q, k, v, out, B, S, P, row_stride, head0, heads, head_dim, sliding_window_size,
+                      num_frame_per_block, num_frame_for_scale, dtype, stream);
 }
 
 // =================================================================== band GQA
@@ -643,24 +679,50 @@ AppendParams append_params(swa_stream* h, int global_idx, int frame_idx, const v
   p.max_pages = h->max_pages;
   p.max_segs = h->max_segs;
   p.copy = 1;
+  p.src_row_bytes = h->row_bytes;
+  p.src_off = 0;
   return p;
+}
+}  // namespace
+
+namespace {
+// Append from k_frame / v_frame whose token rows are row_stride elements apart,
+// the cached heads starting at head ``head0`` of each row.
+swa_status stream_append_impl(swa_stream* h, int global_idx, int frame_idx, const void* k_frame, const void* v_frame,
+                              int64_t row_stride, int head0, void* stream) {
+  swa_status s = stream_check_layer(h, global_idx);
+  if (s != SWA_OK) return s;
+  if (!k_frame || !v_frame || !aligned16(k_frame) || !aligned16(v_frame)) return SWA_ERR_ARG;
+  const int esize = h->cfg.dtype == SWA_F32 ? 4 : 2;
+  if (head0 < 0 || row_stride < static_cast<int64_t>(head0 + h->cfg.heads) * h->cfg.head_dim) return SWA_ERR_SHAPE;
+  if ((row_stride * esize) % 16 != 0 || (static_cast<int64_t>(head0) * h->cfg.head_dim * esize) % 16 != 0)
+    return SWA_ERR_ARG;
+  if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
+  if (frame_idx >= h->cfg.max_frames) return SWA_ERR_CAPACITY;
+  int* err = nullptr;
+  if (const swa_status ds = device_ready(&err)) return ds;
+  AppendParams p = append_params(h, global_idx, frame_idx, k_frame, v_frame, err);
+  p.src_row_bytes = row_stride * esize;
+  p.src_off = static_cast<int64_t>(head0) * h->cfg.head_dim * esize;
+  const cudaError_t e = launch_append_evict(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return SWA_ERR_CUDA;
+  h->n_frames[global_idx] = frame_idx + 1;
+  return SWA_OK;
 }
 }  // namespace
 
 extern "C" swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx, const void* k_frame,
                                               const void* v_frame, void* stream) {
-  swa_status s = stream_check_layer(h, global_idx);
-  if (s != SWA_OK) return s;
-  if (!k_frame || !v_frame || !aligned16(k_frame) || !aligned16(v_frame)) return SWA_ERR_ARG;
-  if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
-  if (frame_idx >= h->cfg.max_frames) return SWA_ERR_CAPACITY;
-  int* err = nullptr;
-  if (const swa_status ds = device_ready(&err)) return ds;
-  const AppendParams p = append_params(h, global_idx, frame_idx, k_frame, v_frame, err);
-  const cudaError_t e = launch_append_evict(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return SWA_ERR_CUDA;
-  h->n_frames[global_idx] = frame_idx + 1;
-  return SWA_OK;
+  if (!h) return SWA_ERR_ARG;
+  return stream_append_impl(h, global_idx, frame_idx, k_frame, v_frame,
+                            static_cast<int64_t>(h->cfg.heads) * h->cfg.head_dim, 0, stream);
+}
+
+extern "C" swa_status swa_stream_append_evict_heads(swa_stream* h, int global_idx, int frame_idx,
+                                                    const void* k_frame, const void* v_frame, int row_stride,
+                                                    int head0, void* stream) {
+  if (!h) return SWA_ERR_ARG;
+  return stream_append_impl(h, global_idx, frame_idx, k_frame, v_frame, row_stride, head0, stream);
 }
 
 // ================================================================ attn_pre prologue
@@ -671,10 +733,22 @@ bool pre_shape_ok(int P, int C, int heads) {
   return (D == 64 || D == 128) && C % 256 == 0 && C <= 2048;  // C % 128: whole feature tiles
 }
 
+// The 3-D RoPE the prologue generates itself (null rot): frame index, special
+// tokens at (t, 0, 0), patch-grid width and frequency base.
+struct RopeGen {
+  int frame, special, grid_w;
+  double theta;
+};
+
+bool rope_gen_ok(const RopeGen& g, int P) {
+  return g.frame >= 0 && g.special >= 0 && g.special <= P && g.grid_w >= 1 && g.theta > 1.0;
+}
+
 swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
                         const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
                         const float* kn_b, const float* rot, int P, int C, int heads, float eps, void* xn_ws,
-                        void* q_out, uint8_t* k_dst, uint8_t* v_dst, cudaStream_t st) {
+                        void* q_out, uint8_t* k_dst, uint8_t* v_dst, cudaStream_t st,
+                        const RopeGen* gen = nullptr) {
   int* err = nullptr;
   if (const swa_status ds = device_ready(&err)) return ds;
   if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
@@ -698,6 +772,22 @@ swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, con
   p.H = heads;
   p.D = C / heads;
   p.eps = eps;
+  if (!rot) {
+    // bands t | h | w of (D/2 - 2*(D/6), D/6, D/6) pairs; pair j of a band of n
+    // pairs turns by pos * theta^(-j/n) (the same rule as swa_rope3d_table)
+    const int half = p.D / 2, n_h = p.D / 6, n_t = half - 2 * n_h;
+    p.rope_frame = gen->frame;
+    p.rope_special = gen->special;
+    p.rope_grid_w = gen->grid_w;
+    p.rope_nt = n_t;
+    p.rope_nh = n_h;
+    const double lt = std::log(gen->theta);
+    for (int j = 0; j < half; ++j) {
+      const int jj = j < n_t ? j : (j < n_t + n_h ? j - n_t : j - n_t - n_h);
+      const int n = j < n_t ? n_t : (j < n_t + n_h ? n_h : half - n_t - n_h);
+      p.rope_inv_freq[j] = std::exp(-lt * jj / n);
+    }
+  }
   return cuda_status(launch_qkv_pre(p, st));
 }
 }  // namespace
@@ -716,6 +806,24 @@ extern "C" swa_status swa_attn_pre(const void* x, const float* ln_w, const float
                       static_cast<uint8_t*>(k_out), static_cast<uint8_t*>(v_out), static_cast<cudaStream_t>(stream));
 }
 
+extern "C" swa_status swa_attn_pre_rope3d(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
+                                          const float* b_qkv, const float* qn_w, const float* qn_b,
+                                          const float* kn_w, const float* kn_b, int frame_idx, int num_special,
+                                          int grid_w, double theta, int P, int C, int heads, float eps,
+                                          void* xn_ws, void* q_out, void* k_out, void* v_out, void* stream) {
+  if (!pre_shape_ok(P, C, heads)) return (P < 0 || heads < 1 || C < 1) ? SWA_ERR_ARG : SWA_ERR_UNSUPPORTED;
+  if (!(eps > 0.f)) return SWA_ERR_ARG;
+  const RopeGen gen{frame_idx, num_special, grid_w, theta};
+  if (!rope_gen_ok(gen, P)) return SWA_ERR_ARG;
+  if (P == 0) return SWA_OK;
+  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, xn_ws, q_out, k_out, v_out};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return SWA_ERR_ARG;
+  return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, nullptr, P, C, heads, eps, xn_ws, q_out,
+                      static_cast<uint8_t*>(k_out), static_cast<uint8_t*>(v_out), static_cast<cudaStream_t>(stream),
+                      &gen);
+}
+
 extern "C" swa_status swa_rope3d_table(int frame_idx, int P, int num_special, int grid_w, int head_dim,
                                        double theta, float* rot_out, void* stream) {
   if (frame_idx < 0 || P < 0 || num_special < 0 || num_special > P || grid_w < 1 || head_dim < 6 ||
@@ -729,11 +837,11 @@ extern "C" swa_status swa_rope3d_table(int frame_idx, int P, int num_special, in
                                          static_cast<cudaStream_t>(stream)));
 }
 
-extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
-                                                  const float* ln_w, const float* ln_b, const void* w_qkv,
-                                                  const float* b_qkv, const float* qn_w, const float* qn_b,
-                                                  const float* kn_w, const float* kn_b, const float* rot, float eps,
-                                                  void* xn_ws, void* q_out, void* stream) {
+namespace {
+swa_status stream_append_pre_impl(swa_stream* h, int global_idx, int frame_idx, const void* x, const float* ln_w,
+                                  const float* ln_b, const void* w_qkv, const float* b_qkv, const float* qn_w,
+                                  const float* qn_b, const float* kn_w, const float* kn_b, const float* rot,
+                                  float eps, void* xn_ws, void* q_out, void* stream, const RopeGen* gen) {
   swa_status s = stream_check_layer(h, global_idx);
   if (s != SWA_OK) return s;
   const swa_stream_cfg& c = h->cfg;
@@ -741,9 +849,11 @@ extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx,
   const int C = c.heads * c.head_dim;
   if (!pre_shape_ok(c.P, C, c.heads)) return SWA_ERR_UNSUPPORTED;
   if (!(eps > 0.f)) return SWA_ERR_ARG;
-  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, xn_ws, q_out};
+  if (gen && !rope_gen_ok(*gen, c.P)) return SWA_ERR_ARG;
+  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, xn_ws, q_out};
   for (const void* q : ptrs)
     if (!q || !aligned16(q)) return SWA_ERR_ARG;
+  if (!gen && (!rot || !aligned16(rot))) return SWA_ERR_ARG;
   if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
   if (frame_idx >= c.max_frames) return SWA_ERR_CAPACITY;
   int* err = nullptr;
@@ -759,8 +869,29 @@ extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx,
                             h->ppf * c.page_tokens;
   uint8_t* kd = layer_k(h, global_idx) + slot_row0 * h->row_bytes;
   uint8_t* vd = layer_v(h, global_idx) + slot_row0 * h->row_bytes;
-  return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot, c.P, C, c.heads, eps, xn_ws,
-                      q_out, kd, vd, st);
+  return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, gen ? nullptr : rot, c.P, C, c.heads,
+                      eps, xn_ws, q_out, kd, vd, st, gen);
+}
+}  // namespace
+
+extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
+                                                  const float* ln_w, const float* ln_b, const void* w_qkv,
+                                                  const float* b_qkv, const float* qn_w, const float* qn_b,
+                                                  const float* kn_w, const float* kn_b, const float* rot, float eps,
+                                                  void* xn_ws, void* q_out, void* stream) {
+  return stream_append_pre_impl(h, global_idx, frame_idx, x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, rot,
+                                eps, xn_ws, q_out, stream, nullptr);
+}
+
+extern "C" swa_status swa_stream_append_evict_pre_rope3d(swa_stream* h, int global_idx, int frame_idx,
+                                                         const void* x, const float* ln_w, const float* ln_b,
+                                                         const void* w_qkv, const float* b_qkv, const float* qn_w,
+                                                         const float* qn_b, const float* kn_w, const float* kn_b,
+                                                         int num_special, int grid_w, double theta, float eps,
+                                                         void* xn_ws, void* q_out, void* stream) {
+  const RopeGen gen{frame_idx, num_special, grid_w, theta};
+  return stream_append_pre_impl(h, global_idx, frame_idx, x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b,
+                                nullptr, eps, xn_ws, q_out, stream, &gen);
 }
 
 namespace {
@@ -788,9 +919,11 @@ namespace {
 // The attend of a frame's queries against key runs listed in device metadata:
 // hdr (n_segs at hdr[5]), run rows and lengths, at most max_segs runs, which
 // cover n_frames_keys full frames plus n_special special tokens.
+// q_frame and out: token rows q_ld elements apart, the layer's heads starting at
+// head q_h0 of each row (q_ld 0: the contiguous [P, heads, head_dim] frame).
 swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame, void* out, cudaStream_t st,
                               const int* hdr, const int* seg_row, const int* seg_len, int max_segs,
-                              int n_frames_keys, int n_special) {
+                              int n_frames_keys, int n_special, int64_t q_ld = 0, int q_h0 = 0) {
   int* err = nullptr;
   if (const swa_status ds = device_ready(&err)) return ds;
   const swa_stream_cfg& c = h->cfg;
@@ -813,6 +946,8 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
     p.D = c.head_dim;
     p.max_segs = max_segs;
     p.scale = 1.f / std::sqrt(static_cast<float>(c.head_dim));
+    p.q_ld = q_ld;
+    p.q_h0 = q_h0;
     return cuda_status(launch_attn_simt(p, st));
   }
   const int T = n_frames_keys * cdiv(c.P, kTileRows) + cdiv(n_special, kTileRows);
@@ -821,7 +956,11 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   const int splits = choose_splits(T, items, c.max_splits, num_sms());
   TcParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tm_q, q_frame, c.head_dim, c.heads, c.P, 1)) return SWA_ERR_CUDA;
+  if (!make_map(&p.tm_q, static_cast<const uint8_t*>(q_frame) + static_cast<size_t>(q_h0) * c.head_dim * 2,
+                c.head_dim, c.heads, c.P, 1, q_ld))
+    return SWA_ERR_CUDA;
+  p.out_ld = q_ld;
+  p.out_h0 = q_h0;
   p.tm_k = h->tm_k[global_idx];
   p.tm_v = h->tm_v[global_idx];
   p.out = out;
@@ -843,18 +982,24 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   p.scale_log2 = scale_log2(c.head_dim);
   cudaError_t e = launch_attn_tc(p, c.head_dim, static_cast<int64_t>(items) * splits, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
-  if (splits > 1) e = launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, c.head_dim, splits, st);
+  if (splits > 1)
+    e = launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, c.head_dim, splits, q_ld, q_h0, st);
   return cuda_status(e);
 }
 }  // namespace
 
-extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
-                                        void* out, void* stream) {
+namespace {
+swa_status stream_attend_heads_impl(swa_stream* h, int global_idx, int frame_idx, const void* q_frame, void* out,
+                                    int64_t row_stride, int head0, void* stream) {
   swa_status s = stream_check_layer(h, global_idx);
   if (s != SWA_OK) return s;
   if (!q_frame || !out || !aligned16(q_frame) || !aligned16(out)) return SWA_ERR_ARG;
-  if (h->n_frames[global_idx] == 0 || frame_idx != h->n_frames[global_idx] - 1) return SWA_ERR_ORDER;
   const swa_stream_cfg& c = h->cfg;
+  const int esize = c.dtype == SWA_F32 ? 4 : 2;
+  if (head0 < 0 || row_stride < static_cast<int64_t>(head0 + c.heads) * c.head_dim) return SWA_ERR_SHAPE;
+  if ((row_stride * esize) % 16 != 0 || (static_cast<int64_t>(head0) * c.head_dim * esize) % 16 != 0)
+    return SWA_ERR_ARG;
+  if (h->n_frames[global_idx] == 0 || frame_idx != h->n_frames[global_idx] - 1) return SWA_ERR_ORDER;
   int* meta = layer_meta(h, global_idx);
   const int off_seg_row = 8 + h->n_slots + h->max_pages;
   const int off_seg_len = off_seg_row + h->max_segs;
@@ -863,7 +1008,21 @@ extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame
   const int n_special =
       c.cross_frame_special ? stream_n_evicted(i, c.scale_frames, c.window_frames) * c.num_special : 0;
   return stream_attend_impl(h, global_idx, q_frame, out, static_cast<cudaStream_t>(stream), meta,
-                            meta + off_seg_row, meta + off_seg_len, h->max_segs, n_ret, n_special);
+                            meta + off_seg_row, meta + off_seg_len, h->max_segs, n_ret, n_special, row_stride, head0);
+}
+}  // namespace
+
+extern "C" swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
+                                        void* out, void* stream) {
+  if (!h) return SWA_ERR_ARG;
+  return stream_attend_heads_impl(h, global_idx, frame_idx, q_frame, out,
+                                  static_cast<int64_t>(h->cfg.heads) * h->cfg.head_dim, 0, stream);
+}
+
+extern "C" swa_status swa_stream_attend_heads(swa_stream* h, int global_idx, int frame_idx, const void* q_frame,
+                                              void* out, int row_stride, int head0, void* stream) {
+  if (!h) return SWA_ERR_ARG;
+  return stream_attend_heads_impl(h, global_idx, frame_idx, q_frame, out, row_stride, head0, stream);
 }
 
 extern "C" swa_status swa_stream_attend_transient(swa_stream* h, int global_idx, const void* q_frame,

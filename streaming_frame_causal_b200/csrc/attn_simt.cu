@@ -31,8 +31,10 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
   const int b = static_cast<int>(gw / (static_cast<int64_t>(p.Hq) * p.Nq));
   const int kvh = h / (p.Hq / p.Hkv);
 
+  const int64_t q_ld = p.q_ld ? p.q_ld : static_cast<int64_t>(p.Hq) * D;
+  const int64_t kv_ld = p.kv_ld ? p.kv_ld : static_cast<int64_t>(p.Hkv) * D;
   float qv[E];
-  const float* qp = p.q + ((static_cast<int64_t>(b) * p.Nq + row) * p.Hq + h) * D;
+  const float* qp = p.q + (static_cast<int64_t>(b) * p.Nq + row) * q_ld + static_cast<int64_t>(p.q_h0 + h) * D;
 #pragma unroll
   for (int e = 0; e < E; ++e) qv[e] = qp[lane + 32 * e] * p.scale;
 
@@ -72,7 +74,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
     const int a = grow ? grow[s] : lo[s];
     const int z = grow ? grow[s] + glen[s] : hi[s];
     for (int key = a; key < z; ++key) {
-      const int64_t koff = ((static_cast<int64_t>(b) * p.Nk + key) * p.Hkv + kvh) * D;
+      const int64_t koff = (static_cast<int64_t>(b) * p.Nk + key) * kv_ld + static_cast<int64_t>(p.kv_h0 + kvh) * D;
       float d = 0.f;
 #pragma unroll
       for (int e = 0; e < E; ++e) d = fmaf(qv[e], p.k[koff + lane + 32 * e], d);
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
       m = m_new;
     }
   }
-  float* op = p.out + ((static_cast<int64_t>(b) * p.Nq + row) * p.Hq + h) * D;
+  float* op = p.out + (static_cast<int64_t>(b) * p.Nq + row) * q_ld + static_cast<int64_t>(p.q_h0 + h) * D;
   const float inv = 1.f / l;
 #pragma unroll
   for (int e = 0; e < E; ++e) op[lane + 32 * e] = o[e] * inv;

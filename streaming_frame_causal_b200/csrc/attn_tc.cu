@@ -218,6 +218,15 @@ SWA_DEV Work decode_work(const TcParams& p) {
 // Measured on B200 (same-box sweeps of 2, 3, 4): 3 is fastest at head_dim 64,
 // where the row sums come from the tensor core and leave the FMA pipe room, and
 // 2 at head_dim 128.  SWA_POLY_PAIRS_D64 / _D128 override them for tuning builds.
+#ifndef SWA_ISSUE_WARP
+#define SWA_ISSUE_WARP 0
+#endif
+// SWA_EX2_BF16X2: at head_dim 64 the MUFU pairs round the exponent argument to
+// bf16 and take 2^x of both halves in one packed instruction (the result is the
+// bf16 P the PV product reads)
+#ifndef SWA_EX2_BF16X2
+#define SWA_EX2_BF16X2 0
+#endif
 #ifndef SWA_POLY_PAIRS_D64
 #define SWA_POLY_PAIRS_D64 3
 #endif
@@ -364,12 +373,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Lane 0 issues every tcgen05.mma.  The issue path is kept short (a
-    // single thread's instruction latency bounds the MMA rate for N <= 128):
-    // shared-memory descriptors are built once, and a K step or a ring stage
-    // moves the start-address field by a constant (addresses stay below 2^18,
-    // so the 14-bit field never carries).
-    if (lane == 0 && T > 0) {
+    // One thread issues every tcgen05.mma and the commits that track them.
+    // With SWA_ISSUE_WARP the whole warp runs the issue loop (uniform control
+    // flow, the descriptors held alike by every lane) and the instructions are
+    // predicated on one elected lane; otherwise lane 0 runs it alone.  The issue
+    // path is kept short (a single thread's instruction latency bounds the MMA
+    // rate for N <= 128): shared-memory descriptors are built once, and a K step
+    // or a ring stage moves the start-address field by a constant (addresses
+    // stay below 2^18, so the 14-bit field never carries).
+#if SWA_ISSUE_WARP
+    const bool run = T > 0;
+    const uint32_t issue = elect_one();
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.err, ERR_WAIT_MMA));
+    };
+#else
+    const bool run = lane == 0 && T > 0;
+    const uint32_t issue = 1;
+    const uint32_t tm = tmem;
+    auto wait = [&](uint32_t bar, uint32_t parity) { return mbar_wait(bar, parity, p.err, ERR_WAIT_MMA); };
+#endif
+    if (run) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, PL::kON, 1);
       constexpr uint64_t kStageStep = PL::kTileBytes >> 4;
@@ -379,11 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       auto issue_qk = [&](int g, int st) {
         const uint64_t dq = dq0 + g * kStageStep;  // Q tiles are kTileBytes apart too
         const uint64_t dk = dk0 + st * kStageStep;
-        const uint32_t tS = tmem + PL::col_s(g);
+        const uint32_t tS = tm + PL::col_s(g);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kSubBytes + (kk & 3) * 32) >> 4);
-          mma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss_if(issue, tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int g, int st, bool acc) {
@@ -391,38 +416,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // leading-byte offset that shrinks as the stage moves up
         const uint64_t dv = PL::kSumCol ? dv0 + st * kStageStep - ((st * kStageStep) << 16)
                                         : dv0 + st * kStageStep;
-        const uint32_t tP = tmem + PL::col_p(g), tO = tmem + PL::col_o(g);
+        const uint32_t tP = tm + PL::col_p(g), tO = tm + PL::col_o(g);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_if(issue, tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(q_full(0), 0, p.err, ERR_WAIT_MMA);
-      if (ok && has_b) ok = mbar_wait(q_full(1), 0, p.err, ERR_WAIT_MMA);
-      if (ok) ok = mbar_wait(k_full(0), 0, p.err, ERR_WAIT_MMA);
+      bool ok = wait(q_full(0), 0);
+      if (ok && has_b) ok = wait(q_full(1), 0);
+      if (ok) ok = wait(k_full(0), 0);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
-        mma_commit(s_full(0));
+        mma_commit_if(issue, s_full(0));
         if (has_b) {
           issue_qk(1, 0);
-          mma_commit(s_full(1));
+          mma_commit_if(issue, s_full(1));
         }
-        if (PL::kSplitKV) mma_commit(k_empty(0));
+        if (PL::kSplitKV) mma_commit_if(issue, k_empty(0));
       }
       const int ng = has_b ? 2 : 1;
       // Fixed order per key tile: PV_A(j) QK_A(j+1) | PV_B(j) QK_B(j+1), each
-      // tile's MMAs back to back with its commit after them.  At head_dim 128
-      // P_g aliases S_g: QK_g(j+1) follows PV_g(j) in this thread's issue
-      // order, which the tensor core keeps.
+      // tile's MMAs back to back with its commit after them.  P_g aliases S_g:
+      // QK_g(j+1) follows PV_g(j) in the issuing thread's order, which the
+      // tensor core keeps.
       for (int j = 0; j < T && ok; ++j) {
         const int st = j % PL::kStages;
         const int st1 = (j + 1) % PL::kStages;
         const bool more = j + 1 < T;
-        if (more && !mbar_wait(k_full(st1), ((j + 1) / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
-        if (PL::kSplitKV && !mbar_wait(v_full(st), (j / PL::kStages) & 1, p.err, ERR_WAIT_MMA)) break;
+        if (more && !wait(k_full(st1), ((j + 1) / PL::kStages) & 1)) break;
+        if (PL::kSplitKV && !wait(v_full(st), (j / PL::kStages) & 1)) break;
 #pragma unroll 1
         for (int g = 0; g < ng; ++g) {
-          if (!mbar_wait(p_full(g), j & 1, p.err, ERR_WAIT_MMA)) {
+          if (!wait(p_full(g), j & 1)) {
             ok = false;
             break;
           }
@@ -430,22 +455,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           issue_pv(g, st, j > 0);
           if (more) {
             issue_qk(g, st1);
-            mma_commit(s_full(g));
+            mma_commit_if(issue, s_full(g));
           } else {
-            mma_commit(o_full(g));
+            mma_commit_if(issue, o_full(g));
           }
         }
         if (!ok) break;
         if (PL::kSplitKV) {
-          mma_commit(v_empty(st));
-          if (more) mma_commit(k_empty(st1));
+          mma_commit_if(issue, v_empty(st));
+          if (more) mma_commit_if(issue, k_empty(st1));
         } else {
-          mma_commit(k_empty(st));  // K_j and V_j leave together after PV_B(j)
+          mma_commit_if(issue, k_empty(st));  // K_j and V_j leave together after PV_B(j)
         }
       }
-      // drain every MMA this thread issued before the CTA may free TMEM
-      mma_commit(drain(0));
-      mbar_wait(drain(0), 0, p.err, ERR_WAIT_MMA);
+      // drain every MMA the issuing thread started before the CTA may free TMEM
+      mma_commit_if(issue, drain(0));
+      wait(drain(0), 0);
     }
   }
   } else {
@@ -567,6 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         float2 pr;
         if ((pi & 7) < kPolyPairs<D>) {
           pr = exp2_poly2(x);
+        } else if (SWA_EX2_BF16X2 && PL::kSumCol) {
+          s[pi] = ex2_bf16x2(pack_bf16x2(x.x, x.y));
+          continue;
         } else {
           pr.x = ex2_approx(x.x);
           pr.y = ex2_approx(x.y);
@@ -605,7 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tmem_wait_ld();
           if (!store) continue;
           if (w.split < 0) {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + idx * D + c0;
+            const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                 (static_cast<int64_t>(w.b) * p.Nq + row) * out_ld +
+                                 static_cast<int64_t>(p.out_h0 + my_h) * D + c0;
 #pragma unroll
             for (int c = 0; c < 32; c += 8) {
               uint4 v;
@@ -656,7 +687,7 @@ template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml,
                                                       __nv_bfloat16* __restrict__ out, int rows,
-                                                      int H, int splits) {
+                                                      int H, int splits, int64_t out_ld, int out_h0) {
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= rows * H) return;
@@ -694,7 +725,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     }
   }
   const float inv = 1.f / L;
-  __nv_bfloat16* dst = out + static_cast<int64_t>(gw) * D + lane * E;
+  const int row = gw / H, h = gw - row * H;
+  __nv_bfloat16* dst = out + static_cast<int64_t>(row) * out_ld + static_cast<int64_t>(out_h0 + h) * D + lane * E;
   if constexpr (E == 2) {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   } else {
@@ -743,15 +775,16 @@ cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cud
 }
 
 cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
-                           int head_dim, int splits, cudaStream_t stream) {
+                           int head_dim, int splits, int64_t out_ld, int out_h0, cudaStream_t stream) {
   const int warps = rows * H;
   const int blocks = (warps + 7) / 8;
   if (blocks == 0) return cudaSuccess;
   auto* o = reinterpret_cast<__nv_bfloat16*>(out);
+  if (out_ld == 0) out_ld = static_cast<int64_t>(H) * head_dim;
   if (head_dim == 64)
-    combine_kernel<64><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits);
+    combine_kernel<64><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits, out_ld, out_h0);
   else if (head_dim == 128)
-    combine_kernel<128><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits);
+    combine_kernel<128><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits, out_ld, out_h0);
   else
     return cudaErrorInvalidValue;
   count_launches(1);

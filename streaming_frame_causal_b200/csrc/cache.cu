@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
       const int64_t sp_row = special_row0 + static_cast<int64_t>(ev - p.S) * p.num_special + row;
       reinterpret_cast<uint4*>(store + sp_row * p.row_bytes)[ch] = *dst;
     }
-    if (p.copy) *dst = reinterpret_cast<const uint4*>(src + static_cast<int64_t>(row) * p.row_bytes)[ch];
+    if (p.copy) *dst = reinterpret_cast<const uint4*>(src + p.src_off + static_cast<int64_t>(row) * p.src_row_bytes)[ch];
   }
 
   if (blockIdx.x != 0) return;

@@ -43,12 +43,15 @@ struct TcParams {
   int W, n_qtiles;           // band mode
   int splits, max_segs;      // stream mode
   float scale_log2;          // log2(e) / sqrt(D)
+  int64_t out_ld;            // elements between consecutive token rows of out (0: Hq * D)
+  int out_h0;                // head of out that query head 0 writes (a head slice of wider rows)
 };
 
 cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream);
 int tc_smem_bytes(int head_dim);
+// out row r, head h at out + r * out_ld + (out_h0 + h) * head_dim (out_ld 0: H * head_dim)
 cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
-                           int head_dim, int splits, cudaStream_t stream);
+                           int head_dim, int splits, int64_t out_ld, int out_h0, cudaStream_t stream);
 
 // ---------------------------------------------------------------- SIMT f32 path
 enum SimtMode : int { SIMT_FRAME = 0, SIMT_BAND = 1, SIMT_STREAM = 2, SIMT_DECODE = 3 };
@@ -69,6 +72,10 @@ struct SimtParams {
   int n_valid;       // decode: valid slots
   int max_segs;
   float scale;
+  int64_t q_ld;      // elements between token rows of q and out (0: Hq * D)
+  int q_h0;          // head of q / out that query head 0 reads and writes
+  int64_t kv_ld;     // elements between token rows of k and v (0: Hkv * D)
+  int kv_h0;         // head of k / v that KV head 0 reads
 };
 
 cudaError_t launch_attn_simt(const SimtParams& p, cudaStream_t stream);
@@ -88,6 +95,8 @@ struct AppendParams {
   int max_pages, max_segs;
   int copy;              // 0: move specials and rewrite metadata only (the frame's K/V
                          // are written into its slot by the attn_pre prologue)
+  int64_t src_row_bytes; // bytes between consecutive tokens of k_src / v_src
+  int64_t src_off;       // byte offset of the cached heads within a source token row
 };
 
 cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream);
@@ -164,6 +173,12 @@ struct PreParams {
   int* err;
   int P, C, H, D;
   float eps;
+  // 3-D RoPE generated in the epilogue when rot is null: token k sits at
+  // (t, h, w) = (rope_frame, (k - s) / rope_grid_w, (k - s) % rope_grid_w) for
+  // k >= s = rope_special and at (rope_frame, 0, 0) below; pair j < rope_nt turns
+  // by t, j < rope_nt + rope_nh by h, the rest by w, times rope_inv_freq[j]
+  int rope_frame, rope_special, rope_grid_w, rope_nt, rope_nh;
+  double rope_inv_freq[64];
 };
 cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
                            cudaStream_t stream);

@@ -108,6 +108,9 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
 }
 
 // ---------------------------------------------------------------- qkv GEMM
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+
 constexpr int kPreThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
 constexpr int kPreM = 128;        // tokens per tile
 constexpr int kPreN = 128;        // output features per tile (2 heads of 64 or 1 of 128)
@@ -223,6 +226,10 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
           v[j + 3] = __uint_as_float(a[j + 3]) + bb.w;
         }
       };
+      // this token's (h, w) grid position for the generated 3-D RoPE
+      const int rope_k = row - p.rope_special;
+      const int rope_h = (p.rot || rope_k < 0) ? 0 : rope_k / p.rope_grid_w;
+      const int rope_w = (p.rot || rope_k < 0) ? 0 : rope_k - rope_h * p.rope_grid_w;
 #pragma unroll 1
       for (int hh = 0; hh < kPreN / D; ++hh) {
         const bool valid = row < p.P;
@@ -263,7 +270,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
               v[j + 2] = (v[j + 2] - mean) * rs * ww.z + bb.z;
               v[j + 3] = (v[j + 3] - mean) * rs * ww.w + bb.w;
             }
-            if (valid) {
+            if (valid && p.rot) {
               // RoPE: pairs (2i, 2i+1) times (cos, sin) of pair i; two pairs per 16-byte load
               const float4* rt = reinterpret_cast<const float4*>(p.rot + static_cast<int64_t>(row) * D + c0);
 #pragma unroll
@@ -274,6 +281,21 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
                 v[j + 1] = x0 * cs.y + x1 * cs.x;
                 v[j + 2] = x2 * cs.z - x3 * cs.w;
                 v[j + 3] = x2 * cs.w + x3 * cs.z;
+              }
+            } else if (valid) {
+              // 3-D RoPE generated here: the pair's angle pos * inv_freq in double,
+              // reduced to [-pi, pi] in double, then sin and cos in float
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const int pair = (c0 + j) >> 1;
+                const int pos = pair < p.rope_nt ? p.rope_frame : (pair < p.rope_nt + p.rope_nh ? rope_h : rope_w);
+                const double ang = static_cast<double>(pos) * p.rope_inv_freq[pair];
+                const double red = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
+                float sn, cs;
+                __sincosf(static_cast<float>(red), &sn, &cs);
+                const float x0 = v[j], x1 = v[j + 1];
+                v[j] = x0 * cs - x1 * sn;
+                v[j + 1] = x0 * sn + x1 * cs;
               }
             }
           }

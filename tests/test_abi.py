@@ -188,3 +188,34 @@ def test_decode_plan_bench_shape_and_bad_args(swa):
     for bad in ((0, 8, 4096, 1), (1, 0, 4096, 1), (1, 8, 0, 1), (1, 8, 4096, -1)):
         with pytest.raises(swa.SwaError):
             swa.swa_sched_decode(*bad)
+
+
+def test_head_slices_and_generated_rope_are_validated(swa):
+    lib = swa._lib
+    # row stride shorter than head0 + heads: rejected before anything runs
+    assert lib.swa_prefill_heads(256, 256, 256, 256, 1, 2, 16, 512, 4, 8, 64, 2, 1, 0, 1, None) == -2
+    # row stride not a multiple of 16 bytes
+    assert lib.swa_prefill_heads(256, 256, 256, 256, 1, 2, 16, 1028, 0, 8, 64, 2, 1, 0, 1, None) == -1
+    # negative head offset
+    assert lib.swa_prefill_heads(256, 256, 256, 256, 1, 2, 16, 1024, -1, 8, 64, 2, 1, 0, 1, None) == -1
+    # generated RoPE: grid width 0, negative frame, theta <= 1, specials beyond P
+    args = [256] * 9
+    for fr, ns, gw, th in ((0, 5, 0, 1e4), (-1, 5, 27, 1e4), (0, 5, 27, 1.0), (0, 2000, 27, 1e4)):
+        assert lib.swa_attn_pre_rope3d(*args, fr, ns, gw, th, 1004, 1024, 16, 1e-6, 256, 256, 256, 256,
+                                       None) == -1
+
+
+def test_binding_argument_counts_match_the_header(swa):
+    """Every ctypes signature the binding declares takes as many arguments as
+    the header's declaration of that function."""
+    import re
+    with open(swa.HEADER_PATH) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    decls = dict((m.group(1), m.group(2)) for m in re.finditer(r"\b(swa_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text))
+    checked = 0
+    for name, (_, args) in swa._sigs.items():
+        params = decls[name].strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert n == len(args), (name, n, len(args))
+        checked += 1
+    assert checked == len(decls)

@@ -128,3 +128,49 @@ def test_rope3d_table_rejects_bad_arguments(swa):
     assert lib.swa_rope3d_table(0, 16, 5, 3, 63, 10000.0, buf.data_ptr(), None) == -1
     assert lib.swa_rope3d_table(0, 16, 5, 3, 64, 1.0, buf.data_ptr(), None) == -1
     assert lib.swa_rope3d_table(0, 16, 5, 3, 64, 10000.0, None, None) == -1
+
+
+@pytest.mark.parametrize("frame,H", [(0, 16), (7, 16), (999, 16), (999, 8)])
+def test_prologue_generates_3d_rope(swa, frame, H):
+    """The lingbot-map frame (5 special tokens + a 37 x 27 grid) with the 3-D RoPE
+    generated inside the prologue: q/k against the oracle's prologue with its
+    float64 table, v unchanged; head_dim 64 and 128."""
+    P, C = 5 + 37 * 27, 1024
+    inp = synth.prologue_inputs(seed=900 + frame + H, P=P, C=C, heads=H)
+    d = {k: v.cuda() for k, v in inp.items()}
+    q, k, v = swa.swa_attn_pre_rope3d(d["x"], *(d[n] for n in ORDER[:-1]), heads=H, frame_idx=frame,
+                                      num_special=5, grid_w=27, eps=EPS)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error_check() == 0
+    a = {n: t.double().numpy() for n, t in inp.items()}
+    a["rot"] = orc.rope3d_table(frame, P, 5, 27, C // H)
+    rq, rk, rv = orc.attn_pre(a["x"], *(a[n] for n in ORDER), heads=H, eps=EPS)
+    for got, ref, name in ((q, rq, "q"), (k, rk, "k"), (v, rv, "v")):
+        check_bf16(got.float().cpu().numpy(), ref, f"{name}, generated 3-D RoPE, frame {frame}")
+
+
+def test_fused_append_with_generated_rope(swa):
+    """The streaming append with the generated 3-D RoPE writes into the slot
+    exactly what swa_attn_pre_rope3d computes for the frame's index."""
+    P, C, H, S, Wc, F = 5 + 37 * 27, 1024, 16, 1, 2, 4
+    D = C // H
+    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
+                          max_frames=F, dtype=torch.bfloat16)
+    ks, vs = cache.storage(0, "k"), cache.storage(0, "v")
+    ppf = -(-P // 16)
+    oc = orc.StreamCache(heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, page_tokens=16,
+                         max_frames=F)
+    for i in range(F):
+        inp = synth.prologue_inputs(seed=70 + i, P=P, C=C, heads=H)
+        d = {k: v.cuda() for k, v in inp.items()}
+        q_ref, k_ref, v_ref = swa.swa_attn_pre_rope3d(d["x"], *(d[n] for n in ORDER[:-1]), heads=H, frame_idx=i,
+                                                      num_special=5, grid_w=27, eps=EPS)
+        q_out = torch.empty_like(q_ref)
+        cache.swa_stream_append_evict_pre_rope3d(0, i, d["x"], *(d[n] for n in ORDER[:-1]), q_out=q_out,
+                                                 num_special=5, grid_w=27, eps=EPS)
+        torch.cuda.synchronize()
+        assert torch.equal(q_out, q_ref)
+        r0 = oc.slot_of(i) * ppf * 16
+        oc.append_evict(0, i, np.zeros((P, H, D)), np.zeros((P, H, D)))
+        assert torch.equal(ks[r0:r0 + P], k_ref) and torch.equal(vs[r0:r0 + P], v_ref)
+    assert swa.swa_device_error_check() == 0
