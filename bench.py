@@ -12,6 +12,11 @@ input, all inputs resident in HBM:
               W = 4096                                               2.062 TFLOP
   * decode    batch 64 at position 200000 against a 4096-slot rolling cache,
               GQA 32/8, head_dim 128 (1 GiB of K/V read)         64 tokens
+Timed apart from the step and reported under ``parts`` as well: the whole
+300-frame stream from an empty cache (fill included, frames/s and per-frame
+latency percentiles), the 1000-frame stream with special-token retention near
+frame 999, the non-keyframe attend, and the attention prologue (with a RoPE
+table and with the 3-D RoPE generated inside it).
 ``value`` is useful attention TFLOP/s over the whole step (visible query-key
 pairs x 4 x head_dim per head; masked and padded work not counted).  Per-stage
 throughput (TFLOP/s, frames/s, decode tokens/s and GB/s) is under ``parts``.
@@ -412,6 +417,20 @@ def run_ours(args, rank, world, local_rank):
         pre_ms = e0.elapsed_time(e1) / n_pre
         parts_out["prologue_us"] = pre_ms * 1e3
         parts_out["prologue_qkv_tflops"] = 2.0 * ST["P"] * Cm * 3 * Cm / (pre_ms * 1e-3) / 1e12
+        # the same prologue with the frame's 3-D RoPE generated inside it (no table)
+        def pre3d():
+            swa.swa_attn_pre_rope3d(pin["x"], *pre_args[:-1], heads=ST["H"], frame_idx=999, num_special=5,
+                                    grid_w=27, q_out=pre_out[0], k_out=pre_out[1], v_out=pre_out[2], xn_ws=pre_ws)
+        for _ in range(3):
+            pre3d()
+        torch.cuda._sleep(50_000_000)
+        e0.record(stream)
+        for _ in range(n_pre):
+            pre3d()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        parts_out["prologue_rope3d_us"] = e0.elapsed_time(e1) / n_pre * 1e3
+        parts_out.update(whole_streams(swa, torch, dev, stream, frames))
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12
         parts_out["band_ms"] = per["band"]
@@ -476,6 +495,75 @@ def run_ours(args, rank, world, local_rank):
         "parts": parts_out, "roofline": roof, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clk,
     }
+    return out
+
+
+def stream_keys(i, S, Wc, P, specials=0):
+    """Keys frame i attends to: retained full frames (scale + window) times P,
+    plus the special tokens kept from evicted frames."""
+    n_full = min(i + 1, S + Wc) if Wc > 0 else i + 1
+    n_evicted = max(0, i + 1 - S - Wc) if Wc > 0 else 0
+    return n_full * P + specials * n_evicted
+
+
+def whole_streams(swa, torch, dev, stream, frames):
+    """Two streams timed apart from the step, append + attend per frame:
+    * the 300-frame stream from an empty cache (fill included): frames/s over
+      all 300 frames and per-frame latency percentiles;
+    * the 1000-frame stream that keeps the 5 special tokens of every evicted
+      frame: frames 0..991 appended (bookkeeping and K/V only), then frames
+      992..999 appended and attended (76,928 keys at frame 999), timed.
+    Frame contents come from the pool of 16 synthetic frames."""
+    out = {}
+    P, H, D, S, Wc = ST["P"], ST["H"], ST["D"], ST["S"], ST["Wc"]
+    sout = torch.empty(P, H, D, dtype=torch.bfloat16, device=dev)
+    n_pool = len(frames)
+    # ---- 300 frames, fill included
+    F = 300
+    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
+                          page_tokens=ST["page"], max_frames=F, max_splits=12, device=dev)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(F + 1)]
+    torch.cuda._sleep(50_000_000)
+    for i in range(F):
+        fq, fk, fv = frames[i % n_pool]
+        evs[i].record(stream)
+        cache.swa_stream_append_evict(0, i, fk, fv)
+        cache.swa_stream_attend(0, i, fq, sout)
+    evs[F].record(stream)
+    torch.cuda.synchronize()
+    lat = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(F))
+    total = evs[0].elapsed_time(evs[F])
+    fl = sum(P * stream_keys(i, S, Wc, P) * H * 4 * D for i in range(F))
+    out["stream300_frames_per_s"] = F / (total * 1e-3)
+    out["stream300_tflops"] = fl / (total * 1e-3) / 1e12
+    out["stream300_frame_ms_p50"] = lat[F // 2]
+    out["stream300_frame_ms_p99"] = lat[min(F - 1, (99 * F) // 100)]
+    cache.close()
+    # ---- 1000 frames with special-token retention, timed near frame 999
+    F = 1000
+    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
+                          page_tokens=ST["page"], cross_frame_special=True, num_special=5, max_frames=F,
+                          max_splits=12, device=dev)
+    t0 = F - 8
+    for i in range(t0):
+        fq, fk, fv = frames[i % n_pool]
+        cache.swa_stream_append_evict(0, i, fk, fv)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(50_000_000)
+    e0.record(stream)
+    for i in range(t0, F):
+        fq, fk, fv = frames[i % n_pool]
+        cache.swa_stream_append_evict(0, i, fk, fv)
+        cache.swa_stream_attend(0, i, fq, sout)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    fl = sum(P * stream_keys(i, S, Wc, P, 5) * H * 4 * D for i in range(t0, F))
+    out["stream1000_special_keys_at_999"] = stream_keys(F - 1, S, Wc, P, 5)
+    out["stream1000_special_ms_per_frame"] = ms / (F - t0)
+    out["stream1000_special_frames_per_s"] = (F - t0) / (ms * 1e-3)
+    out["stream1000_special_tflops"] = fl / (ms * 1e-3) / 1e12
+    cache.close()
     return out
 
 
