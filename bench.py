@@ -7,7 +7,7 @@ input, all inputs resident in HBM:
               frames (schedule + tcgen05 attention)                  1.474 TFLOP
   * stream    8 consecutive frames of a 300-frame-style stream at steady state:
               append + evict on the device, split-KV attend over 8 scale + 64
-              window frames (72 x 1004 keys), combine          8 x 0.297 TFLOP
+              window frames (72 x 1004 keys), merged in-kernel 8 x 0.297 TFLOP
   * band      Mistral-style token window: 32768 tokens, GQA 32/8, head_dim 128,
               W = 4096                                               2.062 TFLOP
   * decode    batch 64 at position 200000 against a 4096-slot rolling cache,
@@ -291,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
         swa.swa_decode(q, k_new, v_new, dkc, dvc, DC["pos"], out, workspace=dws)
 
     def stream_part(frame_evs=None):
-        # frame_evs: events around each frame (append + attend + combine) for
+        # frame_evs: events around each frame (append + attend) for
         # per-frame latency percentiles
         for j in range(ST["frames_per_step"]):
             if frame_evs is not None:
@@ -374,6 +374,7 @@ def run_ours(args, rank, world, local_rank):
                      for j in range(ST["frames_per_step"]))
         parts_out["stream_frame_ms_p50"] = lat[len(lat) // 2]
         parts_out["stream_frame_ms_p99"] = lat[min(len(lat) - 1, (99 * len(lat)) // 100)]
+    if "stream" in per and not args.no_extras:
         # the non-keyframe path at the same steady state (timed apart from the
         # step): the frame attends to the cache plus itself, nothing persists,
         # so its keys are 8 scale + 64 window + 1 frames
@@ -448,7 +449,7 @@ def run_ours(args, rank, world, local_rank):
     # the step.  attn_tc_kernel<64> runs the prefill launch and the eight
     # streaming attends; its launch duration is taken on the prefill launch, the
     # one launch of it that the step brackets alone with CUDA events (a streaming
-    # attend shares its events with the append and combine kernels), and on the
+    # attend shares its events with the append kernel), and on the
     # streaming stage only when the prefill stage is not run.
     cands = []
     if "band" in per:
@@ -460,7 +461,7 @@ def run_ours(args, rank, world, local_rank):
             cands.append((share, per["prefill"], "attn_tc_kernel<64>, prefill launch 32x1004 16x64",
                           flops_prefill(), "attn_tc_prefill_32x1004_h16_d64", "tensor"))
         else:
-            cands.append((share, per["stream"], "attn_tc_kernel<64> stream attend + append + combine, 8 frames",
+            cands.append((share, per["stream"], "attn_tc_kernel<64> stream attend + append, 8 frames",
                           stage_flops["stream"], "attn_tc_stream_72x1004_h16_d64", "tensor"))
     if "decode" in per:
         cands.append((per["decode"], per["decode"], "decode_tc_kernel<4> B64 W4096", decode_bytes(),
@@ -484,8 +485,9 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": recorded_traffic(tkey)}
 
     # ---- end to end through the public API: pinned host inputs -> device -> results back
-    e2e = run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk, bv, bout, dq, dkn, dvn,
-                  dout, frames, sout, prefill, band, decode, stream_frame, world, dist, flops)
+    e2e = None if args.no_extras else run_e2e(args, swa, torch, dev, stream, parts, pq, pk, pv, pout, bq, bk,
+                                               bv, bout, dq, dkn, dvn, dout, frames, sout, prefill, band, decode,
+                                               stream_frame, world, dist, flops)
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -766,6 +768,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", choices=("all", "prefill", "stream", "band", "decode"), default="all",
                     help="time one stage only (for profiling); the reported value then covers that stage")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="run the timed step only: skip the measurements taken apart from it (non-keyframe "
+                         "attend, prologue, whole streams) and the end-to-end pass (for launch lists)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

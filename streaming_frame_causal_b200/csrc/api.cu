@@ -501,6 +501,7 @@ struct swa_stream {
   uint8_t* store0;
   float* part_o;
   float* part_ml;
+  int* split_cnt;  // per attend work item: CTAs of the item that have written their partials
   std::vector<int> n_frames;
   std::vector<CUtensorMap> tm_k, tm_v;
 };
@@ -543,8 +544,11 @@ bool stream_geom(const swa_stream_cfg* c, StreamGeom* g) {
   g->meta_stride = round256(static_cast<size_t>(g->meta_ints + 8 + 2 * (g->max_segs + 1)) * 4);
   g->store_bytes = round256(static_cast<size_t>(g->total_rows) * g->row_bytes);
   const size_t rows_h = static_cast<size_t>(c->P) * c->heads;
+  // split-KV partials (O, then max and sum), then one arrival counter per attend
+  // work item (head x query-tile pair) for the merge in the attend's last CTA
   g->part_bytes = round256(static_cast<size_t>(c->max_splits) * rows_h * c->head_dim * 4) +
-                  round256(static_cast<size_t>(c->max_splits) * rows_h * 2 * 4);
+                  round256(static_cast<size_t>(c->max_splits) * rows_h * 2 * 4) +
+                  round256(static_cast<size_t>(c->heads) * qpairs_per_frame(c->P) * 4);
   g->total = g->meta_stride * c->num_layers + 2 * g->store_bytes * c->num_layers + g->part_bytes;
   return true;
 }
@@ -608,6 +612,8 @@ extern "C" swa_status swa_stream_init(swa_stream** out, const swa_stream_cfg* cf
   h->part_o = reinterpret_cast<float*>(part);
   h->part_ml = reinterpret_cast<float*>(part + round256(static_cast<size_t>(cfg->max_splits) * rows_h *
                                                         cfg->head_dim * 4));
+  h->split_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(h->part_ml) +
+                                        round256(static_cast<size_t>(cfg->max_splits) * rows_h * 2 * 4));
   h->n_frames.assign(cfg->num_layers, 0);
   if (cfg->dtype == SWA_BF16) {
     h->tm_k.resize(cfg->num_layers);
@@ -639,6 +645,8 @@ extern "C" swa_status swa_stream_reset(swa_stream* h, void* stream) {
   // metadata: all -1 (empty slots, no eviction); counters rewritten per append
   cudaError_t e = cudaMemsetAsync(h->meta0, 0xff, h->meta_stride * h->cfg.num_layers, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->store0, 0, 2 * h->store_bytes * h->cfg.num_layers, st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(h->split_cnt, 0, static_cast<size_t>(h->cfg.heads) * qpairs_per_frame(h->cfg.P) * 4, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
   for (int l = 0; l < h->cfg.num_layers; ++l) {
     // header counters start at zero (frames, evicted, specials) and -1 (last evicted)
@@ -966,6 +974,7 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   p.out = out;
   p.part_o = h->part_o;
   p.part_ml = h->part_ml;
+  p.split_cnt = h->split_cnt;
   p.seg_row = seg_row;
   p.seg_len = seg_len;
   p.meta_hdr = hdr;
@@ -982,8 +991,7 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   p.scale_log2 = scale_log2(c.head_dim);
   cudaError_t e = launch_attn_tc(p, c.head_dim, static_cast<int64_t>(items) * splits, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
-  if (splits > 1)
-    e = launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, c.head_dim, splits, q_ld, q_h0, st);
+  // splits > 1: the last CTA of each work item merges the item's partials
   return cuda_status(e);
 }
 }  // namespace

@@ -1,6 +1,7 @@
 // attn_tc.cu -- tcgen05 / TMEM / TMA attention kernel for sm_100a (bf16 in,
 // f32 accumulate, bf16 out), used by the frame-causal prefill, the streaming
-// attend (split-KV with a combine pass) and the token-band GQA prefill.
+// attend (split-KV, merged by the last CTA of each work item) and the
+// token-band GQA prefill.
 //
 // What it computes: O = softmax(Q K^T / sqrt(D)) V over the keys the schedule
 // lists for a 128-row query tile ("Sliding Window Attention Mechanism in
@@ -41,6 +42,14 @@
 #include "ptx.cuh"
 #include "tile_sched.h"
 
+// Build-time variants of the kernel (A/B timing builds):
+#ifndef SWA_ISSUE_WARP
+#define SWA_ISSUE_WARP 1
+#endif
+#ifndef SWA_SRING
+#define SWA_SRING 0
+#endif
+
 namespace swa {
 
 namespace {
@@ -65,7 +74,11 @@ struct Plan {
   // (in f32, from the same bf16 P the PV uses) and is rescaled with O.  The PV
   // then has N = D + 16.  At D = 128 that would not fit tensor memory; the
   // softmax threads add the row sums themselves.
-  static constexpr bool kSumCol = (D == 64);
+  // D = 64 with SWA_SRING: three S buffers in a ring shared by the two query
+  // tiles (the next QK^T of a tile runs while its softmax works on the
+  // current one); the row sums then come from the softmax, O has D columns
+  static constexpr bool kRing = (D == 64) && (SWA_SRING != 0);
+  static constexpr bool kSumCol = (D == 64) && !kRing;
   // K and V stages with their own barriers (released after the QK^T and after
   // the PV respectively) for the two-stage ring at head_dim 128; one barrier per
   // stage for both at head_dim 64, where the four-stage ring has slack and the
@@ -78,7 +91,7 @@ struct Plan {
   // that reads P, and tcgen05.mma operations from one thread execute in issue order.
   SWA_DEV static uint32_t col_s(int g) { return g ? 128u : 0u; }
   SWA_DEV static uint32_t col_p(int g) { return col_s(g); }
-  SWA_DEV static uint32_t col_o(int g) { return g ? 384u : 256u; }
+  SWA_DEV static uint32_t col_o(int g) { return kRing ? 384u + 64u * g : (g ? 384u : 256u); }
   static constexpr uint32_t kTmemCols = 512;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
@@ -86,8 +99,8 @@ struct Plan {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffOnes = kOffV + kStages * kTileBytes;  // the constant block (kSumCol)
   static constexpr int kOffBar = kOffOnes + (kSumCol ? kSubBytes : 0);
-  static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 2;
-  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kNumBars = 2 + 4 * kStages + 3 + 2 + 2 + 2 + 2;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;   // TMEM base (4 bytes), then the merge flag
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
 };
 
@@ -218,15 +231,6 @@ SWA_DEV Work decode_work(const TcParams& p) {
 // Measured on B200 (same-box sweeps of 2, 3, 4): 3 is fastest at head_dim 64,
 // where the row sums come from the tensor core and leave the FMA pipe room, and
 // 2 at head_dim 128.  SWA_POLY_PAIRS_D64 / _D128 override them for tuning builds.
-#ifndef SWA_ISSUE_WARP
-#define SWA_ISSUE_WARP 0
-#endif
-// SWA_EX2_BF16X2: at head_dim 64 the MUFU pairs round the exponent argument to
-// bf16 and take 2^x of both halves in one packed instruction (the result is the
-// bf16 P the PV product reads)
-#ifndef SWA_EX2_BF16X2
-#define SWA_EX2_BF16X2 0
-#endif
 #ifndef SWA_POLY_PAIRS_D64
 #define SWA_POLY_PAIRS_D64 3
 #endif
@@ -268,10 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   auto k_empty = [&](int s) { return bar0 + 8u * (2 + 2 * PL::kStages + s); };
   auto v_empty = [&](int s) { return bar0 + 8u * (2 + 3 * PL::kStages + s); };
   constexpr int kB = 2 + 4 * PL::kStages;
-  auto s_full = [&](int g) { return bar0 + 8u * (kB + g); };
-  auto p_full = [&](int g) { return bar0 + 8u * (kB + 2 + g); };
-  auto o_full = [&](int g) { return bar0 + 8u * (kB + 4 + g); };
-  auto drain = [&](int g) { return bar0 + 8u * (kB + 6 + g); };
+  auto s_full = [&](int i) { return bar0 + 8u * (kB + i); };      // per S buffer (3 in the ring)
+  auto p_full = [&](int g) { return bar0 + 8u * (kB + 3 + g); };
+  auto o_full = [&](int g) { return bar0 + 8u * (kB + 5 + g); };
+  auto drain = [&](int g) { return bar0 + 8u * (kB + 7 + g); };
+  auto o_done = [&](int g) { return bar0 + 8u * (kB + 9 + g); };  // ring: PV_g(j) complete
   const uint32_t tmem_slot = base + PL::kOffTmem;
 
   if (threadIdx.x == 0) {
@@ -285,6 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     mbar_init(s_full(0), 1);
     mbar_init(s_full(1), 1);
+    mbar_init(s_full(2), 1);
+    mbar_init(o_done(0), 1);
+    mbar_init(o_done(1), 1);
     mbar_init(p_full(0), 128);
     mbar_init(p_full(1), 128);
     for (int g = 0; g < 2; ++g) {
@@ -424,6 +432,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = wait(q_full(0), 0);
       if (ok && has_b) ok = wait(q_full(1), 0);
       if (ok) ok = wait(k_full(0), 0);
+      if constexpr (PL::kRing) {
+        // QK^T ops in the order A0 B0 A1 B1 A2 ...: op n of the sequence (n =
+        // 2j + g, or j with one tile) writes S buffer n mod 3, whose previous
+        // user, op n - 3, had its PV issued before it (P aliases its S)
+        auto seq = [&](int g, int j) { return has_b ? 2 * j + g : j; };
+        auto qk_ring = [&](int g, int j) {
+          const int n = seq(g, j);
+          const uint64_t dq = dq0 + g * kStageStep;
+          const uint64_t dk = dk0 + (j % PL::kStages) * kStageStep;
+          const uint32_t tS = tm + 128u * static_cast<uint32_t>(n % 3);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kSubBytes + (kk & 3) * 32) >> 4);
+            mma_ss_if(issue, tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit_if(issue, s_full(n % 3));
+        };
+        auto pv_ring = [&](int g, int j) {
+          const int st = j % PL::kStages;
+          const uint64_t dv = dv0 + st * kStageStep;
+          const uint32_t tP = tm + 128u * static_cast<uint32_t>(seq(g, j) % 3), tO = tm + PL::col_o(g);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ts_if(issue, tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_if(issue, o_done(g));
+          if (j == T - 1) mma_commit_if(issue, o_full(g));
+        };
+        if (ok) {
+          tc_fence_after();
+          qk_ring(0, 0);
+          if (has_b) qk_ring(1, 0);
+          if (T > 1) {
+            ok = wait(k_full(1 % PL::kStages), (1 / PL::kStages) & 1);
+            if (ok) qk_ring(0, 1);
+          }
+        }
+        for (int j = 0; j < T && ok; ++j) {
+          if (!wait(p_full(0), j & 1)) break;
+          tc_fence_after();
+          pv_ring(0, j);
+          if (has_b) {
+            if (j + 1 < T) qk_ring(1, j + 1);
+            if (!wait(p_full(1), j & 1)) break;
+            tc_fence_after();
+            pv_ring(1, j);
+          }
+          mma_commit_if(issue, k_empty(j % PL::kStages));  // K_j and V_j leave after the last PV(j)
+          if (j + 2 < T) {
+            if (!wait(k_full((j + 2) % PL::kStages), ((j + 2) / PL::kStages) & 1)) break;
+            qk_ring(0, j + 2);
+          }
+        }
+        ok = false;  // the fixed-order loop below is for the other layouts
+      }
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -480,8 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + PL::col_s(g);
-    const uint32_t tP = tmem + lane_off + PL::col_p(g);
+    const uint32_t tS0 = tmem + lane_off + PL::col_s(g);
     const uint32_t tO = tmem + lane_off + PL::col_o(g);
     const float sl2 = p.scale_log2;
     const bool band = (p.mode == TC_BAND);
@@ -503,7 +564,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int krow, kvalid;
       cursor_tile(w, cur, &krow, &kvalid);
       cursor_next(w, cur);
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), j & 1, p.err, ERR_WAIT_SOFTMAX))) {
+      // this key tile's S buffer and the phase of its barrier
+      int sbuf = g;
+      uint32_t sphase = j & 1;
+      if constexpr (PL::kRing) {
+        const int n = has_b ? 2 * j + g : j;
+        sbuf = n % 3;
+        sphase = (n / 3) & 1;
+      }
+      const uint32_t tS = PL::kRing ? tmem + lane_off + 128u * static_cast<uint32_t>(sbuf) : tS0;
+      const uint32_t tP = tS;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(sbuf), sphase, p.err, ERR_WAIT_SOFTMAX))) {
         ok = false;
         break;
       }
@@ -554,8 +625,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         m = m_new;
       }
       if (__any_sync(0xffffffffu, grow)) {
-        // O of this tile is complete up to key tile j-1 (the commit that
-        // signalled S_j covers the earlier PV), so it can be rescaled in place
+        // O of this tile must be complete up to key tile j-1 before it is
+        // rescaled in place: the commit that signalled S_j covers the earlier
+        // PV, except in the ring, where PV(j-1) may still run (wait for it)
+        if (PL::kRing && j > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(o_done(g), (j - 1) & 1, p.err, ERR_WAIT_SOFTMAX))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t orr[32];
@@ -592,9 +671,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         float2 pr;
         if ((pi & 7) < kPolyPairs<D>) {
           pr = exp2_poly2(x);
-        } else if (SWA_EX2_BF16X2 && PL::kSumCol) {
-          s[pi] = ex2_bf16x2(pack_bf16x2(x.x, x.y));
-          continue;
         } else {
           pr.x = ex2_approx(x.x);
           pr.y = ex2_approx(x.y);
@@ -661,11 +737,67 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < my_rows) {
-      // empty split: contributes nothing to the combine
+      // empty split: contributes nothing to the merge
       const int row = my_row0 + r;
       const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
       p.part_ml[idx * 2 + 0] = -INFINITY;
       p.part_ml[idx * 2 + 1] = 0.f;
+    }
+    if (w.split >= 0) {
+      // ---- split-KV merge in the item's last CTA: every thread publishes its
+      // partial stores (fence), the 256 softmax threads meet, one of them
+      // counts this CTA in; the CTA that completes the count merges all of the
+      // item's partials, O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c (m
+      // in log2 units), and puts the count back for the next launch
+      volatile int* flag = reinterpret_cast<volatile int*>(gbase + PL::kOffTmem + 8);
+      const int item = static_cast<int>(blockIdx.x % (static_cast<unsigned>(p.Hq) * p.n_pairs));
+      __threadfence();
+      __syncwarp();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (warp == 4 && lane == 0) *flag = (atomicAdd(p.split_cnt + item, 1) == p.splits - 1) ? 1 : 0;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (*flag) {
+        __threadfence();
+        if ((g == 0 || has_b) && r < my_rows) {
+          const int row = my_row0 + r;
+          const int64_t stride = static_cast<int64_t>(p.Nq) * p.Hq;
+          const int64_t base_idx = static_cast<int64_t>(row) * p.Hq + my_h;
+          float M = -INFINITY;
+          for (int c = 0; c < p.splits; ++c) M = fmaxf(M, __ldcg(p.part_ml + (c * stride + base_idx) * 2));
+          float L = 0.f;
+          float o[D];
+#pragma unroll
+          for (int e = 0; e < D; ++e) o[e] = 0.f;
+          for (int c = 0; c < p.splits; ++c) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (c * stride + base_idx) * 2));
+            const float wc = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+            L = fmaf(wc, ml.y, L);
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + (c * stride + base_idx) * D);
+#pragma unroll
+            for (int e = 0; e < D / 4; ++e) {
+              const float4 v = __ldcg(src + e);
+              o[4 * e] = fmaf(wc, v.x, o[4 * e]);
+              o[4 * e + 1] = fmaf(wc, v.y, o[4 * e + 1]);
+              o[4 * e + 2] = fmaf(wc, v.z, o[4 * e + 2]);
+              o[4 * e + 3] = fmaf(wc, v.w, o[4 * e + 3]);
+            }
+          }
+          const float inv = 1.f / L;
+          const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * out_ld +
+                               static_cast<int64_t>(p.out_h0 + my_h) * D;
+#pragma unroll
+          for (int e = 0; e < D; e += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+            v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+            v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+            v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + e) = v;
+          }
+        }
+        if (warp == 4 && lane == 0) p.split_cnt[item] = 0;
+      }
     }
   }
 
@@ -675,65 +807,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, PL::kTmemCols);
-  }
-}
-
-// ---------------------------------------------------------------- combine
-// O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c  (m in log2 units), the
-// log-sum-exp merge of split-KV partials.  One warp per (row, head): lane c
-// holds split c's (m, l), the warp reduces M and the weighted sum, then every
-// lane accumulates its slice of O over the splits with independent loads.
-template <int D>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part_o,
-                                                      const float* __restrict__ part_ml,
-                                                      __nv_bfloat16* __restrict__ out, int rows,
-                                                      int H, int splits, int64_t out_ld, int out_h0) {
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (gw >= rows * H) return;
-  const int64_t stride = static_cast<int64_t>(rows) * H;
-  float mc = -INFINITY, lc = 0.f;
-  if (lane < splits) {
-    const float2 ml = *reinterpret_cast<const float2*>(part_ml + (lane * stride + gw) * 2);
-    mc = ml.x;
-    lc = ml.y;
-  }
-  float M = mc;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  const float wc = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-  float L = wc * lc;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-  constexpr int E = D / 32;  // elements per lane: 2 (D = 64) or 4 (D = 128)
-  float acc[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  for (int c = 0; c < splits; ++c) {
-    const float w = __shfl_sync(0xffffffffu, wc, c);
-    const float* src = part_o + (c * stride + gw) * D + lane * E;
-    if constexpr (E == 2) {
-      const float2 v = *reinterpret_cast<const float2*>(src);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-    } else {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-    }
-  }
-  const float inv = 1.f / L;
-  const int row = gw / H, h = gw - row * H;
-  __nv_bfloat16* dst = out + static_cast<int64_t>(row) * out_ld + static_cast<int64_t>(out_h0 + h) * D + lane * E;
-  if constexpr (E == 2) {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  } else {
-    uint2 v;
-    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(dst) = v;
   }
 }
 
@@ -772,23 +845,6 @@ cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cud
   if (head_dim == 64) return launch_tc_d<64>(p, n_items, stream);
   if (head_dim == 128) return launch_tc_d<128>(p, n_items, stream);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
-                           int head_dim, int splits, int64_t out_ld, int out_h0, cudaStream_t stream) {
-  const int warps = rows * H;
-  const int blocks = (warps + 7) / 8;
-  if (blocks == 0) return cudaSuccess;
-  auto* o = reinterpret_cast<__nv_bfloat16*>(out);
-  if (out_ld == 0) out_ld = static_cast<int64_t>(H) * head_dim;
-  if (head_dim == 64)
-    combine_kernel<64><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits, out_ld, out_h0);
-  else if (head_dim == 128)
-    combine_kernel<128><<<blocks, 256, 0, stream>>>(part_o, part_ml, o, rows, H, splits, out_ld, out_h0);
-  else
-    return cudaErrorInvalidValue;
-  count_launches(1);
-  return cudaGetLastError();
 }
 
 }  // namespace swa

@@ -43,15 +43,15 @@ struct TcParams {
   int W, n_qtiles;           // band mode
   int splits, max_segs;      // stream mode
   float scale_log2;          // log2(e) / sqrt(D)
+  int* split_cnt;            // stream mode, splits > 1: per work item (head, query-tile pair),
+                             // CTAs that have written their partials; the last one merges
+                             // them into out and puts the count back to 0
   int64_t out_ld;            // elements between consecutive token rows of out (0: Hq * D)
   int out_h0;                // head of out that query head 0 writes (a head slice of wider rows)
 };
 
 cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream);
 int tc_smem_bytes(int head_dim);
-// out row r, head h at out + r * out_ld + (out_h0 + h) * head_dim (out_ld 0: H * head_dim)
-cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H,
-                           int head_dim, int splits, int64_t out_ld, int out_h0, cudaStream_t stream);
 
 // ---------------------------------------------------------------- SIMT f32 path
 enum SimtMode : int { SIMT_FRAME = 0, SIMT_BAND = 1, SIMT_STREAM = 2, SIMT_DECODE = 3 };

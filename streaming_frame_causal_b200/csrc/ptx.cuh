@@ -290,13 +290,6 @@ SWA_DEV float ex2_approx(float x) {
   return y;
 }
 
-// 2^x of both halves of a bf16 pair on the MUFU unit (inputs and results bf16)
-SWA_DEV uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 SWA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

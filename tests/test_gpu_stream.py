@@ -27,7 +27,7 @@ def _compare_meta(meta, oc, layer, i):
 
 
 def _stream(swa, F, P, H, D, S, Wc, special, dtype, frames_to_check, max_frames=None, layers=1,
-            check_rows=None, num_special=5):
+            check_rows=None, num_special=5, check_heads=None):
     max_frames = max_frames or F
     dev = "cuda"
     cache = swa.SwaStream(num_layers=layers, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc,
@@ -47,7 +47,13 @@ def _stream(swa, F, P, H, D, S, Wc, special, dtype, frames_to_check, max_frames=
                 cache.swa_stream_attend(layer, i, q.to(dev), out)
                 torch.cuda.synchronize()
                 got = out.float().cpu().numpy()
-                if check_rows is None:
+                if check_heads is not None:
+                    # every query row of the listed heads
+                    kc, vc = oc.gather(layer)
+                    qq = q.float().numpy()
+                    ref = np.stack([orc.softmax_attention(qq[:, h], kc[:, h], vc[:, h]) for h in check_heads], 1)
+                    got = got[:, check_heads]
+                elif check_rows is None:
                     ref = oc.attend(layer, q.float().numpy())
                 else:
                     kc, vc = oc.gather(layer)
@@ -145,10 +151,13 @@ def test_300_frame_stream(swa):
 
 
 def test_1000_frame_stream_with_specials(swa):
-    """Same cache, 1000 frames, evicted frames keep 5 special tokens each."""
-    rows = np.unique(np.concatenate([np.arange(0, 1004, 53), [0, 4, 5, 1003]]))
+    """Same cache, 1000 frames, evicted frames keep 5 special tokens each.  Every
+    query row of heads 0 and 15 is checked where the special run changes shape:
+    frame 72 (the first eviction, 5 specials), 73, 75 (20 specials: the run
+    first spills onto a second 16-token page), 87 (80 specials: the run first
+    ends exactly on a page boundary), 500 and 999 (4640 specials, 76,928 keys)."""
     _stream(swa, F=1000, P=1004, H=16, D=64, S=8, Wc=64, special=True, dtype=torch.bfloat16,
-            frames_to_check={72, 500, 999}, check_rows=rows)
+            frames_to_check={72, 73, 75, 87, 500, 999}, check_heads=[0, 15])
 
 
 # ---------------------------------------------------------------- non-keyframe attend
