@@ -49,6 +49,9 @@
 #ifndef SWA_SRING
 #define SWA_SRING 0
 #endif
+#ifndef SWA_PSTORE_SPLIT
+#define SWA_PSTORE_SPLIT 0
+#endif
 
 namespace swa {
 
@@ -666,6 +669,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int pi = 0; pi < 64; ++pi) {
+        // SWA_PSTORE_SPLIT: the first 32 packed pairs go to TMEM while the
+        // second half is computed (pairs 0..31 are final once pi reaches 32)
+        if (SWA_PSTORE_SPLIT && pi == 32) tmem_st32(tP + 0, s);
         const float2 x =
             __ffma2_rn(make_float2(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])), c2, nb2);
         float2 pr;
@@ -680,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       if constexpr (!PL::kSumCol)
         l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-      tmem_st32(tP + 0, s);
+      if (!SWA_PSTORE_SPLIT) tmem_st32(tP + 0, s);
       tmem_st32(tP + 32, s + 32);
       tmem_wait_st();
       tc_fence_before();
@@ -765,35 +771,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           float M = -INFINITY;
           for (int c = 0; c < p.splits; ++c) M = fmaxf(M, __ldcg(p.part_ml + (c * stride + base_idx) * 2));
           float L = 0.f;
-          float o[D];
-#pragma unroll
-          for (int e = 0; e < D; ++e) o[e] = 0.f;
           for (int c = 0; c < p.splits; ++c) {
             const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (c * stride + base_idx) * 2));
-            const float wc = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-            L = fmaf(wc, ml.y, L);
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + (c * stride + base_idx) * D);
-#pragma unroll
-            for (int e = 0; e < D / 4; ++e) {
-              const float4 v = __ldcg(src + e);
-              o[4 * e] = fmaf(wc, v.x, o[4 * e]);
-              o[4 * e + 1] = fmaf(wc, v.y, o[4 * e + 1]);
-              o[4 * e + 2] = fmaf(wc, v.z, o[4 * e + 2]);
-              o[4 * e + 3] = fmaf(wc, v.w, o[4 * e + 3]);
-            }
+            L = fmaf((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M), ml.y, L);
           }
           const float inv = 1.f / L;
           const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * out_ld +
                                static_cast<int64_t>(p.out_h0 + my_h) * D;
+          // 32 output columns at a time, each the weighted sum over the splits
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
 #pragma unroll
-          for (int e = 0; e < D; e += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
-            v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
-            v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
-            v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
-            *reinterpret_cast<uint4*>(dst + e) = v;
+            for (int e = 0; e < 32; ++e) o[e] = 0.f;
+            for (int c = 0; c < p.splits; ++c) {
+              const float m_c = __ldcg(p.part_ml + (c * stride + base_idx) * 2);
+              const float wc = (m_c == -INFINITY) ? 0.f : exp2f(m_c - M);
+              const float4* src = reinterpret_cast<const float4*>(p.part_o + (c * stride + base_idx) * D + c0);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 v = __ldcg(src + e);
+                o[4 * e] = fmaf(wc, v.x, o[4 * e]);
+                o[4 * e + 1] = fmaf(wc, v.y, o[4 * e + 1]);
+                o[4 * e + 2] = fmaf(wc, v.z, o[4 * e + 2]);
+                o[4 * e + 3] = fmaf(wc, v.w, o[4 * e + 3]);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+              v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+              v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+              v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + c0 + e) = v;
+            }
           }
         }
         if (warp == 4 && lane == 0) p.split_cnt[item] = 0;
