@@ -12,7 +12,8 @@
 // CTA organisation (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q tiles once, then K key tiles into a ring (and
 //               at head_dim 64 the V tile of the same key tile beside it)
-//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
+//   warp 1      TMEM allocator; the whole warp runs the MMA issue loop and one
+//               elected lane issues every tcgen05.mma and commit
 //   warp 2      idle
 //   warp 3      TMA producer at head_dim 128: V key tiles into a second ring
 //   warps 4-7   softmax for query tile A (one thread per query row)
@@ -23,11 +24,13 @@
 // The two query tiles ping-pong: while softmax A turns S_A into P_A, the tensor
 // core runs P_B V and Q_B K^T, and the other way round.  S (f32, 128 columns),
 // P (bf16 pairs, 64 columns written over the front of S once it is read) and O
-// (f32, D columns, plus the row-sum column at head_dim 64) of each tile live in
-// tensor memory; P feeds the PV product straight from TMEM (A operand), so the
-// shared-memory operands are Q, K and V, staged by TMA with 128-byte swizzle
-// (and at head_dim 64 a constant block that turns one PV column into the row
-// sum).
+// (f32, D columns) of each tile live in tensor memory; P feeds the PV product
+// straight from TMEM (A operand), so the shared-memory operands are Q, K and V,
+// staged by TMA with 128-byte swizzle.  At head_dim 64 three S buffers form a
+// ring shared by the two tiles: QK^T number n of the sequence A0 B0 A1 B1 ...
+// writes buffer n mod 3 as soon as the PV of op n-3 (whose P sits there) is
+// issued, so a tile's next scores are computed while its softmax still works on
+// the current ones.  At head_dim 128 each tile has one S buffer.
 // Online softmax uses exp2 with the scale folded in and skips rescaling O
 // unless the running maximum grows by more than 2^8 (exact after the final
 // division by the row sum).
@@ -42,21 +45,19 @@
 #include "ptx.cuh"
 #include "tile_sched.h"
 
-// Build-time variants of the kernel (A/B timing builds):
+// Build options, kept for same-box A/B timing against the layouts they replaced
+// (SWA_NVCC_FLAGS="-DSWA_ISSUE_WARP=0" etc. with build.py):
+//   SWA_ISSUE_WARP  1: the whole issuer warp runs the MMA loop, one elected lane
+//                   issues; 0: lane 0 alone runs it
+//   SWA_SRING       1: head_dim 64 uses three S buffers in a ring (below); 0: one
+//                   S buffer per query tile and the row sums from the tensor core
 #ifndef SWA_ISSUE_WARP
 #define SWA_ISSUE_WARP 1
 #endif
 #ifndef SWA_SRING
-#define SWA_SRING 0
+#define SWA_SRING 1
 #endif
-// SWA_KEY_HALVES: head_dim 64 runs attn_hs_kernel (two softmax warpgroups per
-// query tile, one per 64-key half of every key tile)
-#ifndef SWA_KEY_HALVES
-#define SWA_KEY_HALVES 0
-#endif
-#ifndef SWA_PSTORE_SPLIT
-#define SWA_PSTORE_SPLIT 0
-#endif
+
 
 namespace swa {
 
@@ -674,9 +675,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int pi = 0; pi < 64; ++pi) {
-        // SWA_PSTORE_SPLIT: the first 32 packed pairs go to TMEM while the
-        // second half is computed (pairs 0..31 are final once pi reaches 32)
-        if (SWA_PSTORE_SPLIT && pi == 32) tmem_st32(tP + 0, s);
         const float2 x =
             __ffma2_rn(make_float2(__uint_as_float(s[2 * pi]), __uint_as_float(s[2 * pi + 1])), c2, nb2);
         float2 pr;
@@ -691,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       if constexpr (!PL::kSumCol)
         l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-      if (!SWA_PSTORE_SPLIT) tmem_st32(tP + 0, s);
+      tmem_st32(tP + 0, s);
       tmem_st32(tP + 32, s + 32);
       tmem_wait_st();
       tc_fence_before();
@@ -828,478 +826,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
-// ---------------------------------------------------------------- head_dim 64, key halves
-// The same attention at head_dim 64 with twice the softmax warps and no more
-// tensor memory: every 128-key tile's scores are split between two
-// warpgroups, one per 64-key half.  Each half keeps its own running maximum,
-// row sum and O accumulator (the PV of a half multiplies that half's P by that
-// half's 64 rows of V into its own O), so the two halves of a row never
-// exchange anything per tile; the epilogue merges them like two split-KV
-// partials.  640 threads = 5 warpgroups:
-//   warpgroup 0   warp 0 TMA producer (Q once, K and V of a key tile under one
-//                 barrier), warp 1 TMEM allocator and MMA issuer (whole warp,
-//                 one elected lane), warps 2-3 idle
-//   warpgroups 1-4  softmax of (tile A, keys 0-63), (A, 64-127), (B, 0-63),
-//                 (B, 64-127): one thread per query row, 64 scores
-// Tensor memory: S_A 0-127, S_B 128-255 (each half's P over the front of its
-// own 64 columns), O_A0 256, O_A1 320, O_B0 384, O_B1 448 (64 columns each).
-namespace hs {
-constexpr int kThreads = 640;
-constexpr int kRegsLaunch = 96;    // 640 x 96 = 61440 of 65536
-constexpr int kRegsCtl = 64;       // warpgroup 0 after setmaxnreg.dec
-constexpr int kRegsSoftmax = 104;  // warpgroups 1-4 after setmaxnreg.inc
-static_assert(4 * kRegsCtl + 16 * kRegsSoftmax <= 20 * kRegsLaunch,
-              "register split must fit the pool the CTA was launched with");
-constexpr int kStages = 4;
-constexpr int kTileBytes = kRows * 64 * 2;  // 16 KB: a Q, K or V tile
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + 2 * kTileBytes;
-constexpr int kOffV = kOffK + kStages * kTileBytes;
-constexpr int kOffX = kOffV + kStages * kTileBytes;  // epilogue exchange: [tile][half][row] (m, l)
-constexpr int kOffBar = kOffX + 2 * 2 * kRows * 8;
-// q_full 2, kv_full 4, kv_empty 4, s_full 2, p_full 4 (tile x half), o_full 2, drain 1
-constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
-constexpr int kOffTmem = kOffBar + kNumBars * 8;  // TMEM base (4 bytes), then the merge flag
-constexpr int kSmemBytes = kOffTmem + 16 + 1024;
-}  // namespace hs
-
-__global__ void __launch_bounds__(hs::kThreads, 1) attn_hs_kernel(const __grid_constant__ TcParams p) {
-  constexpr int D = 64;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_base = smem_u32(smem_raw);
-  const uint32_t base = (raw_base + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw_base);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  const Work w = decode_work(p);
-  const int T = w.t_end - w.t_begin;
-  const bool has_b = w.rows1 > 0;
-
-  const uint32_t bar0 = base + hs::kOffBar;
-  auto q_full = [&](int g) { return bar0 + 8u * g; };
-  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + hs::kStages + s); };
-  constexpr int kB = 2 + 2 * hs::kStages;
-  auto s_full = [&](int g) { return bar0 + 8u * (kB + g); };
-  auto p_full = [&](int g, int h) { return bar0 + 8u * (kB + 2 + 2 * g + h); };
-  auto o_full = [&](int g) { return bar0 + 8u * (kB + 6 + g); };
-  const uint32_t drain = bar0 + 8u * (kB + 8);
-  const uint32_t tmem_slot = base + hs::kOffTmem;
-
-  if (threadIdx.x == 0) {
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(q_full(g), 1);
-      mbar_init(s_full(g), 1);
-      mbar_init(o_full(g), 1);
-      mbar_init(p_full(g, 0), 128);
-      mbar_init(p_full(g, 1), 128);
-    }
-    for (int s = 0; s < hs::kStages; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
-    }
-    mbar_init(drain, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + hs::kOffTmem);
-  if (warp < 4) {
-    reg_dealloc<hs::kRegsCtl>();
-    if (warp == 0) {
-      // ---------------------------------------------------------- producer
-      if (lane == 0 && T > 0) {
-        tma_prefetch_desc(&p.tm_q);
-        tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_v);
-        for (int g = 0; g < (has_b ? 2 : 1); ++g) {
-          mbar_arrive_expect_tx(q_full(g), hs::kTileBytes);
-          tma_load_4d(base + hs::kOffQ + g * hs::kTileBytes, &p.tm_q, q_full(g), 0, g ? w.h1 : w.h0,
-                      g ? w.qrow1 : w.qrow0, w.b);
-        }
-        Cursor cur;
-        bool ok = cursor_seek(w, w.t_begin, cur);
-        if (!ok) latch_error(p.err, ERR_BAD_META);
-        int issued = 0;
-        for (int j = 0; j < T && ok; ++j) {
-          const int st = j % hs::kStages;
-          if (j >= hs::kStages &&
-              !mbar_wait(kv_empty(st), ((j / hs::kStages) - 1) & 1, p.err, ERR_WAIT_TMA))
-            break;
-          if (cur.s >= w.nseg) {
-            latch_error(p.err, ERR_BAD_META);
-            break;
-          }
-          int krow, kvalid;
-          cursor_tile(w, cur, &krow, &kvalid);
-          mbar_arrive_expect_tx(kv_full(st), 2 * hs::kTileBytes);
-          tma_load_4d(base + hs::kOffK + st * hs::kTileBytes, &p.tm_k, kv_full(st), 0, w.kvh, krow, w.b);
-          tma_load_4d(base + hs::kOffV + st * hs::kTileBytes, &p.tm_v, kv_full(st), 0, w.kvh, krow, w.b);
-          cursor_next(w, cur);
-          ++issued;
-        }
-        // never leave the CTA with a bulk copy still writing its shared memory
-        for (int j = issued - hs::kStages; j < issued; ++j)
-          if (j >= 0) mbar_wait(kv_full(j % hs::kStages), (j / hs::kStages) & 1, p.err, ERR_WAIT_TMA);
-        for (int g = 0; g < (has_b ? 2 : 1); ++g) mbar_wait(q_full(g), 0, p.err, ERR_WAIT_TMA);
-      }
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
-      // Per key tile j and query tile g: PV of key half 0 once its P is in, PV
-      // of half 1 once its P is in, then QK^T(j+1) into S_g (after both PVs
-      // that read P from S_g, in this thread's issue order).
-      const uint32_t issue = elect_one();
-      const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-      auto wait = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.err, ERR_WAIT_MMA));
-      };
-      if (T > 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, 1);
-        constexpr uint64_t kStageStep = hs::kTileBytes >> 4;
-        const uint64_t dq0 = sdesc_sw128(base + hs::kOffQ, 16, 1024);
-        const uint64_t dk0 = sdesc_sw128(base + hs::kOffK, 16, 1024);
-        const uint64_t dv0 = sdesc_sw128(base + hs::kOffV, kSubBytes, 1024);
-        auto issue_qk = [&](int g, int st) {
-          const uint64_t dq = dq0 + g * kStageStep;
-          const uint64_t dk = dk0 + st * kStageStep;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss_if(issue, tm + 128u * g, dq + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-        };
-        auto issue_pv = [&](int g, int h, int st, bool acc) {
-          const uint64_t dv = dv0 + st * kStageStep + ((64 * h * 128) >> 4);
-          const uint32_t tP = tm + 128u * g + 64u * h, tO = tm + 256u + 128u * g + 64u * h;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts_if(issue, tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        };
-        const int ng = has_b ? 2 : 1;
-        bool ok = wait(q_full(0), 0);
-        if (ok && has_b) ok = wait(q_full(1), 0);
-        if (ok) ok = wait(kv_full(0), 0);
-        if (ok) {
-          tc_fence_after();
-          for (int g = 0; g < ng; ++g) {
-            issue_qk(g, 0);
-            mma_commit_if(issue, s_full(g));
-          }
-        }
-        for (int j = 0; j < T && ok; ++j) {
-          const int st = j % hs::kStages;
-          const int st1 = (j + 1) % hs::kStages;
-          const bool more = j + 1 < T;
-          if (more && !wait(kv_full(st1), ((j + 1) / hs::kStages) & 1)) break;
-#pragma unroll 1
-          for (int g = 0; g < ng && ok; ++g) {
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-              if (!wait(p_full(g, h), j & 1)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              issue_pv(g, h, st, j > 0);
-            }
-            if (!ok) break;
-            if (more) {
-              issue_qk(g, st1);
-              mma_commit_if(issue, s_full(g));
-            } else {
-              mma_commit_if(issue, o_full(g));
-            }
-          }
-          if (!ok) break;
-          mma_commit_if(issue, kv_empty(st));  // K_j and V_j leave after the last PV(j)
-        }
-        // drain every MMA the issuing thread started before the CTA may free TMEM
-        mma_commit_if(issue, drain);
-        wait(drain, 0);
-      }
-    }
-  } else {
-    reg_alloc<hs::kRegsSoftmax>();
-    // ------------------------------------------------------------ softmax
-    const int wg = (warp - 4) >> 2;  // 0..3
-    const int g = wg >> 1;           // query tile
-    const int hf = wg & 1;           // key half
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 128u * g + 64u * hf;  // this half's scores; its P over their front
-    const uint32_t tO = tmem + lane_off + 256u + 128u * g + 64u * hf;
-    const float sl2 = p.scale_log2;
-    const bool band = (p.mode == TC_BAND);
-    const int my_h = g ? w.h1 : w.h0;
-    const int my_row0 = g ? w.qrow1 : w.qrow0;
-    const int my_rows = g ? w.rows1 : w.rows0;
-    const int qrow = my_row0 + r;
-    float m = -INFINITY;  // running reference max of this half's raw scores
-    float l = 0.f;        // running row sum of this half relative to m
-    bool ok = (g == 0 || has_b) && T > 0;
-    const bool active = ok;
-    Cursor cur;
-    if (ok) ok = cursor_seek(w, w.t_begin, cur);
-    for (int j = 0; j < T && ok; ++j) {
-      if (cur.s >= w.nseg) {
-        ok = false;
-        break;
-      }
-      int krow, kvalid;
-      cursor_tile(w, cur, &krow, &kvalid);
-      cursor_next(w, cur);
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), j & 1, p.err, ERR_WAIT_SOFTMAX))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // ---- masks: unused tail of the last tile of a key run, band edges.  The
-      // scores are read from TMEM twice, 32 columns at a time (for the row max,
-      // then for the exponentials), so a thread holds 32 of them at once
-      const int kbase = krow + 64 * hf;  // key of this half's column 0
-      const int hvalid = kvalid - 64 * hf;
-      bool full_cols = hvalid >= 64;
-      int lo_key = -0x7fffffff, hi_key = 0x7fffffff;
-      if (band) {
-        const bool inside = (kbase >= my_row0 + my_rows - 1 - p.W + 1) && (kbase + 63 <= my_row0) && hvalid >= 64;
-        if (!inside) {
-          full_cols = false;
-          lo_key = qrow - p.W + 1;
-          hi_key = qrow;
-        }
-      }
-      auto mask32 = [&](uint32_t* v, int c0) {
-        if (full_cols) return;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int key = kbase + c0 + c;
-          if (c0 + c >= hvalid || key < lo_key || key > hi_key) v[c] = __float_as_uint(-INFINITY);
-        }
-      };
-      float a[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) a[k] = -INFINITY;
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tS + c0, v);
-        tmem_wait_ld();
-        mask32(v, c0);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          a[k] = max3f(a[k], max3f(__uint_as_float(v[k]), __uint_as_float(v[8 + k]), __uint_as_float(v[16 + k])),
-                       __uint_as_float(v[24 + k]));
-      }
-      const float tmax = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-      const float m_new = fmaxf(m, tmax);
-      const bool grow = (m != -INFINITY) && ((m_new - m) * sl2 > 8.0f);
-      float alpha = 1.f;
-      if (m == -INFINITY) {
-        m = m_new;
-      } else if (grow) {
-        alpha = ex2_approx((m - m_new) * sl2);
-        m = m_new;
-      }
-      if (__any_sync(0xffffffffu, grow)) {
-        // this half's O is complete up to key tile j-1 (the commit that
-        // signalled S_j covers both halves' earlier PVs): rescale in place
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t orr[32];
-          tmem_ld32(tO + c0, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(tO + c0, orr);
-        }
-        tmem_wait_st();
-      }
-      l *= alpha;
-      // ---- P = 2^(s*scale - m*scale): 32 scores at a time, 16 packed bf16 pairs
-      // stored over the front of this half's (already read) score columns
-      const float nb = (m == -INFINITY) ? 0.f : -m * sl2;
-      const float2 c2 = make_float2(sl2, sl2);
-      const float2 nb2 = make_float2(nb, nb);
-      float2 acc[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tS + c0, v);
-        tmem_wait_ld();
-        mask32(v, c0);
-        uint32_t pk[16];
-#pragma unroll
-        for (int pi = 0; pi < 16; ++pi) {
-          const float2 x =
-              __ffma2_rn(make_float2(__uint_as_float(v[2 * pi]), __uint_as_float(v[2 * pi + 1])), c2, nb2);
-          float2 pr;
-          if ((pi & 7) < kPolyPairs<64>) {
-            pr = exp2_poly2(x);
-          } else {
-            pr.x = ex2_approx(x.x);
-            pr.y = ex2_approx(x.y);
-          }
-          acc[pi & 3] = __fadd2_rn(acc[pi & 3], pr);
-          pk[pi] = pack_bf16x2(pr.x, pr.y);
-        }
-        tmem_st16(tS + c0 / 2, pk);
-      }
-      l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full(g, hf));
-    }
-    // ---- epilogue: merge the two key halves of each row, then store
-    float2* xch = reinterpret_cast<float2*>(gbase + hs::kOffX);  // [g][hf][row]
-    float M = -INFINITY, a_self = 0.f, a_other = 0.f, L = 0.f;
-    const bool have = active && ok &&
-                      __all_sync(0xffffffffu, mbar_wait(o_full(g), 0, p.err, ERR_WAIT_EPI));
-    if (have) xch[(g * 2 + hf) * kRows + r] = make_float2(m == -INFINITY ? -INFINITY : m * sl2, l);
-    // the two warpgroups of this tile meet (named barrier 2 + g, 256 threads)
-    __syncwarp();
-    if (g == 0)
-      asm volatile("bar.sync 2, 256;" ::: "memory");
-    else
-      asm volatile("bar.sync 3, 256;" ::: "memory");
-    if (have) {
-      const float2 mine = xch[(g * 2 + hf) * kRows + r];
-      const float2 other = xch[(g * 2 + (hf ^ 1)) * kRows + r];
-      M = fmaxf(mine.x, other.x);
-      a_self = (mine.x == -INFINITY) ? 0.f : exp2f(mine.x - M);
-      a_other = (other.x == -INFINITY) ? 0.f : exp2f(other.x - M);
-      L = a_self * mine.y + a_other * other.y;
-      tc_fence_after();
-      // this half's thread writes output columns [32 hf, 32 hf + 32) of its row,
-      // 16 at a time
-      const uint32_t tO0 = tmem + lane_off + 256u + 128u * g;  // O of key half 0; half 1 at +64
-      const float w0 = hf ? a_other : a_self;
-      const float w1 = hf ? a_self : a_other;
-      const bool store = r < my_rows;
-      const int row = my_row0 + r;
-      const float inv = 1.f / L;
-      const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
-      const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
-#pragma unroll 1
-      for (int c0 = 32 * hf; c0 < 32 * hf + 32; c0 += 16) {
-        uint32_t o0[16], o1[16];
-        tmem_ld16(tO0 + c0, o0);
-        tmem_ld16(tO0 + 64 + c0, o1);
-        tmem_wait_ld();
-        float f[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) f[e] = w0 * __uint_as_float(o0[e]) + w1 * __uint_as_float(o1[e]);
-        if (store && w.split < 0) {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                               (static_cast<int64_t>(w.b) * p.Nq + row) * out_ld +
-                               static_cast<int64_t>(p.out_h0 + my_h) * D + c0;
-#pragma unroll
-          for (int e = 0; e < 16; e += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(f[e] * inv, f[e + 1] * inv);
-            v.y = pack_bf16x2(f[e + 2] * inv, f[e + 3] * inv);
-            v.z = pack_bf16x2(f[e + 4] * inv, f[e + 5] * inv);
-            v.w = pack_bf16x2(f[e + 6] * inv, f[e + 7] * inv);
-            *reinterpret_cast<uint4*>(dst + e) = v;
-          }
-        } else if (store) {
-          // split-KV partial of the row: the merged numerator relative to M
-          float* dst = p.part_o + idx * D + c0;
-#pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
-        }
-      }
-      if (store && w.split >= 0 && hf == 0) {
-        p.part_ml[idx * 2 + 0] = M;
-        p.part_ml[idx * 2 + 1] = L;
-      }
-    } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < my_rows && hf == 0) {
-      // empty split: contributes nothing to the merge
-      const int row = my_row0 + r;
-      const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
-      p.part_ml[idx * 2 + 0] = -INFINITY;
-      p.part_ml[idx * 2 + 1] = 0.f;
-    }
-    if (w.split >= 0) {
-      // ---- split-KV merge in the item's last CTA (as in attn_tc_kernel): the
-      // 512 softmax threads meet, one counts this CTA in, and the CTA that
-      // completes the count merges the item's partials; each half's threads
-      // take 32 of the 64 output columns of their row
-      volatile int* flag = reinterpret_cast<volatile int*>(gbase + hs::kOffTmem + 8);
-      const int item = static_cast<int>(blockIdx.x % (static_cast<unsigned>(p.Hq) * p.n_pairs));
-      __threadfence();
-      __syncwarp();
-      asm volatile("bar.sync 1, 512;" ::: "memory");
-      if (warp == 4 && lane == 0) *flag = (atomicAdd(p.split_cnt + item, 1) == p.splits - 1) ? 1 : 0;
-      asm volatile("bar.sync 1, 512;" ::: "memory");
-      if (*flag) {
-        __threadfence();
-        if ((g == 0 || has_b) && r < my_rows) {
-          const int row = my_row0 + r;
-          const int64_t stride = static_cast<int64_t>(p.Nq) * p.Hq;
-          const int64_t base_idx = static_cast<int64_t>(row) * p.Hq + my_h;
-          float Mx = -INFINITY;
-          for (int c = 0; c < p.splits; ++c) Mx = fmaxf(Mx, __ldcg(p.part_ml + (c * stride + base_idx) * 2));
-          float Lx = 0.f;
-          for (int c = 0; c < p.splits; ++c) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (c * stride + base_idx) * 2));
-            Lx = fmaf((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - Mx), ml.y, Lx);
-          }
-          const float inv = 1.f / Lx;
-          const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * out_ld +
-                               static_cast<int64_t>(p.out_h0 + my_h) * D;
-#pragma unroll 1
-          for (int c0 = 32 * hf; c0 < 32 * hf + 32; c0 += 16) {
-            float o[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = 0.f;
-            for (int c = 0; c < p.splits; ++c) {
-              const float m_c = __ldcg(p.part_ml + (c * stride + base_idx) * 2);
-              const float wc = (m_c == -INFINITY) ? 0.f : exp2f(m_c - Mx);
-              const float4* src = reinterpret_cast<const float4*>(p.part_o + (c * stride + base_idx) * D + c0);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float4 v = __ldcg(src + e);
-                o[4 * e] = fmaf(wc, v.x, o[4 * e]);
-                o[4 * e + 1] = fmaf(wc, v.y, o[4 * e + 1]);
-                o[4 * e + 2] = fmaf(wc, v.z, o[4 * e + 2]);
-                o[4 * e + 3] = fmaf(wc, v.w, o[4 * e + 3]);
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 16; e += 8) {
-              uint4 v;
-              v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
-              v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
-              v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
-              v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + c0 + e) = v;
-            }
-          }
-        }
-        if (warp == 4 && lane == 0) p.split_cnt[item] = 0;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 }  // namespace
 
 int tc_smem_bytes(int head_dim) {
@@ -1330,27 +856,8 @@ cudaError_t launch_tc_d(const TcParams& p, int64_t n_items, cudaStream_t stream)
 }
 }  // namespace
 
-cudaError_t launch_hs(const TcParams& p, int64_t n_items, cudaStream_t stream) {
-  static DeviceOnce attr_set;  // devices on which the smem opt-in was set
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (!attr_set.done(dev)) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_hs_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs * 20 < 4 * hs::kRegsCtl + 16 * hs::kRegsSoftmax) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(attn_hs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, hs::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set.mark(dev);
-  }
-  attn_hs_kernel<<<static_cast<unsigned>(n_items), hs::kThreads, hs::kSmemBytes, stream>>>(p);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
-  if (head_dim == 64 && SWA_KEY_HALVES) return launch_hs(p, n_items, stream);
   if (head_dim == 64) return launch_tc_d<64>(p, n_items, stream);
   if (head_dim == 128) return launch_tc_d<128>(p, n_items, stream);
   return cudaErrorInvalidValue;
