@@ -15,9 +15,8 @@ input, all inputs resident in HBM:
 Timed apart from the step and reported under ``parts`` as well: the whole
 300-frame stream from an empty cache (fill included, frames/s and per-frame
 latency percentiles), the 1000-frame stream with special-token retention near
-frame 999, the non-keyframe attend, and the attention prologue (two kernels
-with a RoPE table or with the 3-D RoPE generated inside; one kernel with norm1
-folded into the GEMM on prepared weights, both RoPE forms).
+frame 999, the non-keyframe attend, and the attention prologue (with a RoPE
+table and with the 3-D RoPE generated inside it).
 ``value`` is useful attention TFLOP/s over the whole step (visible query-key
 pairs x 4 x head_dim per head; masked and padded work not counted).  Per-stage
 throughput (TFLOP/s, frames/s, decode tokens/s and GB/s) is under ``parts``.
@@ -432,26 +431,6 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         parts_out["prologue_rope3d_us"] = e0.elapsed_time(e1) / n_pre * 1e3
-        # norm1 folded into the GEMM on weights prepared once (one kernel per frame),
-        # with the RoPE table and with the 3-D RoPE generated inside
-        prep = swa.swa_attn_pre_prepare(pin["ln_w"], pin["ln_b"], pin["w_qkv"], pin["b_qkv"])
-        fold_args = [pin[n] for n in ("qn_w", "qn_b", "kn_w", "kn_b")]
-        for name, kw in (("prologue_folded_us", dict(rot=pin["rot"])),
-                         ("prologue_folded_rope3d_us", dict(frame_idx=999, num_special=5, grid_w=27))):
-            def pref():
-                swa.swa_attn_pre_prepared(pin["x"], prep, *fold_args, heads=ST["H"], q_out=pre_out[0],
-                                          k_out=pre_out[1], v_out=pre_out[2], **kw)
-            for _ in range(3):
-                pref()
-            torch.cuda._sleep(50_000_000)
-            e0.record(stream)
-            for _ in range(n_pre):
-                pref()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            parts_out[name] = e0.elapsed_time(e1) / n_pre * 1e3
-        parts_out["prologue_folded_qkv_tflops"] = (2.0 * ST["P"] * Cm * 3 * Cm /
-                                                   (parts_out["prologue_folded_us"] * 1e-6) / 1e12)
         parts_out.update(whole_streams(swa, torch, dev, stream, frames))
     if "band" in per:
         parts_out["band_tflops"] = flops_band() / (per["band"] * 1e-3) / 1e12

@@ -298,42 +298,6 @@ swa_status swa_stream_append_evict_pre_rope3d(swa_stream* h, int global_idx, int
                                               const float* kn_w, const float* kn_b, int num_special, int grid_w,
                                               double theta, float eps, void* xn_ws, void* q_out, void* stream);
 
-/* The attention prologue with norm1 folded into the qkv GEMM, on weights prepared
- * once per weight set.  The prologue's first two steps equal
- *   norm1(x) w_qkv^T + b_qkv = rs * (x W'^T - mu * u) + v,
- *   W' = w_qkv diag(ln_w),  u[n] = sum_c W'[n, c],  v = ln_b w_qkv^T + b_qkv,
- * for a token with mean mu and inverse deviation rs = 1/sqrt(var + eps), so the
- * GEMM reads the raw tokens and no normalised copy goes through device memory;
- * the kernel's epilogue warps take each token's sum and sum of squares from the
- * token tiles as they pass through shared memory.  (Numerically x W'^T is formed
- * before the mean is subtracted: inputs whose mean is many orders of magnitude
- * above their spread lose precision that the two-step path keeps.)
- *
- * swa_attn_pre_weights_bytes: bytes of the prepared weights for C features (0
- * for an unsupported C): W' [3C, C] bf16, then u and v [3C] f32, each at a
- * 256-byte boundary.
- * swa_attn_pre_prepare: writes them into ``prep`` (device, caller-owned, 16-byte
- * aligned) from ln_w, ln_b [C], w_qkv [3C, C] bf16 and b_qkv [3C]; u sums the
- * rounded bf16 W' the GEMM multiplies.  Errors: SWA_ERR_ARG, SWA_ERR_UNSUPPORTED.
- * swa_attn_pre_prepared: the prologue of one frame from x [P, C] bf16 and
- * ``prep``; rot [P, head_dim/2, 2] as in swa_attn_pre, or NULL to generate the
- * 3-D RoPE of (frame_idx, num_special, grid_w, theta) as swa_attn_pre_rope3d does.
- * Outputs and errors as swa_attn_pre.
- * swa_stream_append_evict_pre_prepared: swa_stream_append_evict_pre on prepared
- * weights (rot NULL: the 3-D RoPE of frame ``frame_idx`` generated inside). */
-size_t swa_attn_pre_weights_bytes(int C);
-swa_status swa_attn_pre_prepare(const float* ln_w, const float* ln_b, const void* w_qkv, const float* b_qkv,
-                                int C, void* prep, void* stream);
-swa_status swa_attn_pre_prepared(const void* x, const void* prep, const float* qn_w, const float* qn_b,
-                                 const float* kn_w, const float* kn_b, const float* rot, int frame_idx,
-                                 int num_special, int grid_w, double theta, int P, int C, int heads, float eps,
-                                 void* q_out, void* k_out, void* v_out, void* stream);
-swa_status swa_stream_append_evict_pre_prepared(swa_stream* h, int global_idx, int frame_idx, const void* x,
-                                                const void* prep, const float* qn_w, const float* qn_b,
-                                                const float* kn_w, const float* kn_b, const float* rot,
-                                                int num_special, int grid_w, double theta, float eps,
-                                                void* q_out, void* stream);
-
 /* Layout of one layer's metadata block, in int32 units. */
 typedef struct swa_meta_layout {
     int n_ints;          /* size of the block                                  */

@@ -86,11 +86,6 @@ _sigs = {
     "swa_attn_pre_rope3d": (_i, [_vp] * 9 + [_i, _i, _i, C.c_double, _i, _i, _i, C.c_float] + [_vp] * 5),
     "swa_stream_append_evict_pre_rope3d": (_i, [_vp, _i, _i] + [_vp] * 9 + [_i, _i, C.c_double, C.c_float]
                                            + [_vp] * 3),
-    "swa_attn_pre_weights_bytes": (_sz, [_i]),
-    "swa_attn_pre_prepare": (_i, [_vp] * 4 + [_i, _vp, _vp]),
-    "swa_attn_pre_prepared": (_i, [_vp] * 7 + [_i, _i, _i, C.c_double, _i, _i, _i, C.c_float] + [_vp] * 4),
-    "swa_stream_append_evict_pre_prepared": (_i, [_vp, _i, _i] + [_vp] * 7 + [_i, _i, C.c_double, C.c_float]
-                                             + [_vp, _vp]),
     "swa_stream_meta_layout": (_i, [_vp, C.POINTER(swa_meta_layout)]),
     "swa_stream_get_meta": (_i, [_vp, _i, C.POINTER(swa_meta_host), _vp]),
     "swa_stream_get_meta_raw": (_i, [_vp, _i, _vp, _sz, _vp]),
@@ -248,36 +243,6 @@ def swa_attn_pre_rope3d(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, hea
                                     int(grid_w), float(theta), P, Cdim, heads, float(eps), _ptr(xn_ws),
                                     _ptr(q_out), _ptr(k_out), _ptr(v_out), _stream(stream)),
            "swa_attn_pre_rope3d")
-    return q_out, k_out, v_out
-
-
-def swa_attn_pre_prepare(ln_w, ln_b, w_qkv, b_qkv, out=None, stream=None) -> torch.Tensor:
-    """Prepared weights of the norm1-folded prologue (uint8 device tensor of
-    swa_attn_pre_weights_bytes(C) bytes; layout in include/swa.h)."""
-    Cdim = w_qkv.shape[1]
-    n = int(_lib.swa_attn_pre_weights_bytes(Cdim))
-    if n == 0:
-        raise SwaError(-7, "swa_attn_pre_weights_bytes")
-    out = torch.empty(n, dtype=torch.uint8, device=w_qkv.device) if out is None else out
-    _check(_lib.swa_attn_pre_prepare(_ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv), Cdim, _ptr(out),
-                                     _stream(stream)), "swa_attn_pre_prepare")
-    return out
-
-
-def swa_attn_pre_prepared(x, prep, qn_w, qn_b, kn_w, kn_b, heads: int, rot=None, frame_idx: int = 0,
-                          num_special: int = 0, grid_w: int = 1, theta: float = 10000.0, eps: float = 1e-6,
-                          q_out=None, k_out=None, v_out=None, stream=None):
-    """The prologue of one frame on prepared weights (norm1 folded into the GEMM);
-    rot None generates the frame's 3-D RoPE (see include/swa.h)."""
-    P, Cdim = x.shape
-    D = Cdim // heads
-    q_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if q_out is None else q_out
-    k_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if k_out is None else k_out
-    v_out = torch.empty(P, heads, D, dtype=x.dtype, device=x.device) if v_out is None else v_out
-    _check(_lib.swa_attn_pre_prepared(_ptr(x), _ptr(prep), _ptr(qn_w), _ptr(qn_b), _ptr(kn_w), _ptr(kn_b),
-                                      _ptr(rot), int(frame_idx), int(num_special), int(grid_w), float(theta), P,
-                                      Cdim, heads, float(eps), _ptr(q_out), _ptr(k_out), _ptr(v_out),
-                                      _stream(stream)), "swa_attn_pre_prepared")
     return q_out, k_out, v_out
 
 
@@ -453,17 +418,6 @@ class SwaStream:
             self.handle, global_idx, frame_idx, _ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_qkv), _ptr(b_qkv),
             _ptr(qn_w), _ptr(qn_b), _ptr(kn_w), _ptr(kn_b), int(num_special), int(grid_w), float(theta),
             float(eps), _ptr(xn_ws), _ptr(q_out), _stream(stream)), "swa_stream_append_evict_pre_rope3d")
-        return q_out
-
-    def swa_stream_append_evict_pre_prepared(self, global_idx: int, frame_idx: int, x, prep, qn_w, qn_b, kn_w,
-                                             kn_b, q_out, rot=None, num_special: int = 0, grid_w: int = 1,
-                                             theta: float = 10000.0, eps: float = 1e-6, stream=None):
-        """swa_stream_append_evict_pre on prepared weights (rot None: the frame's
-        3-D RoPE generated inside; see include/swa.h)."""
-        _check(_lib.swa_stream_append_evict_pre_prepared(
-            self.handle, global_idx, frame_idx, _ptr(x), _ptr(prep), _ptr(qn_w), _ptr(qn_b), _ptr(kn_w),
-            _ptr(kn_b), _ptr(rot), int(num_special), int(grid_w), float(theta), float(eps), _ptr(q_out),
-            _stream(stream)), "swa_stream_append_evict_pre_prepared")
         return q_out
 
     def swa_stream_attend_transient(self, global_idx: int, q_frame, k_frame, v_frame, out, stream=None):

@@ -752,28 +752,18 @@ bool rope_gen_ok(const RopeGen& g, int P) {
   return g.frame >= 0 && g.special >= 0 && g.special <= P && g.grid_w >= 1 && g.theta > 1.0;
 }
 
-// prep non-null: norm1 folded into the GEMM with the prepared weights of
-// swa_attn_pre_prepare (ln_w, ln_b, w_qkv, b_qkv and xn_ws are then unused)
 swa_status run_attn_pre(const void* x, const float* ln_w, const float* ln_b, const void* w_qkv,
                         const float* b_qkv, const float* qn_w, const float* qn_b, const float* kn_w,
                         const float* kn_b, const float* rot, int P, int C, int heads, float eps, void* xn_ws,
                         void* q_out, uint8_t* k_dst, uint8_t* v_dst, cudaStream_t st,
-                        const RopeGen* gen = nullptr, const void* prep = nullptr) {
+                        const RopeGen* gen = nullptr) {
   int* err = nullptr;
   if (const swa_status ds = device_ready(&err)) return ds;
+  if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
   PreParams p;
   std::memset(&p, 0, sizeof(p));
-  if (prep) {
-    const size_t wbytes = (static_cast<size_t>(3) * C * C * 2 + 255) & ~static_cast<size_t>(255);
-    p.fold_u = reinterpret_cast<const float*>(static_cast<const uint8_t*>(prep) + wbytes);
-    p.fold_v = p.fold_u + (((static_cast<size_t>(3) * C * 4 + 255) & ~static_cast<size_t>(255)) / 4);
-    if (!encode_2d_sw128(&p.tm_a, x, C, P, 128) || !encode_2d_sw128(&p.tm_b, prep, C, 3LL * C, 128))
-      return SWA_ERR_CUDA;
-  } else {
-    if (launch_ln_rows(x, ln_w, ln_b, xn_ws, P, C, eps, st) != cudaSuccess) return SWA_ERR_CUDA;
-    if (!encode_2d_sw128(&p.tm_a, xn_ws, C, P, 128) || !encode_2d_sw128(&p.tm_b, w_qkv, C, 3LL * C, 128))
-      return SWA_ERR_CUDA;
-  }
+  if (!encode_2d_sw128(&p.tm_a, xn_ws, C, P, 128) || !encode_2d_sw128(&p.tm_b, w_qkv, C, 3LL * C, 128))
+    return SWA_ERR_CUDA;
   p.b_qkv = b_qkv;
   p.qn_w = qn_w;
   p.qn_b = qn_b;
@@ -842,40 +832,6 @@ extern "C" swa_status swa_attn_pre_rope3d(const void* x, const float* ln_w, cons
                       &gen);
 }
 
-extern "C" size_t swa_attn_pre_weights_bytes(int C) {
-  if (C < 256 || C % 256 || C > 2048) return 0;
-  return attn_pre_weights_bytes(C);
-}
-
-extern "C" swa_status swa_attn_pre_prepare(const float* ln_w, const float* ln_b, const void* w_qkv,
-                                           const float* b_qkv, int C, void* prep, void* stream) {
-  if (C < 256 || C % 256 || C > 2048) return SWA_ERR_UNSUPPORTED;
-  const void* ptrs[] = {ln_w, ln_b, w_qkv, b_qkv, prep};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return SWA_ERR_ARG;
-  int* err = nullptr;
-  if (const swa_status ds = device_ready(&err)) return ds;
-  return cuda_status(launch_attn_pre_prepare(ln_w, ln_b, w_qkv, b_qkv, C, prep, static_cast<cudaStream_t>(stream)));
-}
-
-extern "C" swa_status swa_attn_pre_prepared(const void* x, const void* prep, const float* qn_w, const float* qn_b,
-                                            const float* kn_w, const float* kn_b, const float* rot, int frame_idx,
-                                            int num_special, int grid_w, double theta, int P, int C, int heads,
-                                            float eps, void* q_out, void* k_out, void* v_out, void* stream) {
-  if (!pre_shape_ok(P, C, heads)) return (P < 0 || heads < 1 || C < 1) ? SWA_ERR_ARG : SWA_ERR_UNSUPPORTED;
-  if (!(eps > 0.f)) return SWA_ERR_ARG;
-  const RopeGen gen{frame_idx, num_special, grid_w, theta};
-  if (!rot && !rope_gen_ok(gen, P)) return SWA_ERR_ARG;
-  if (P == 0) return SWA_OK;
-  const void* ptrs[] = {x, prep, qn_w, qn_b, kn_w, kn_b, q_out, k_out, v_out};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return SWA_ERR_ARG;
-  if (rot && !aligned16(rot)) return SWA_ERR_ARG;
-  return run_attn_pre(x, nullptr, nullptr, nullptr, nullptr, qn_w, qn_b, kn_w, kn_b, rot, P, C, heads, eps, nullptr,
-                      q_out, static_cast<uint8_t*>(k_out), static_cast<uint8_t*>(v_out),
-                      static_cast<cudaStream_t>(stream), rot ? nullptr : &gen, prep);
-}
-
 extern "C" swa_status swa_rope3d_table(int frame_idx, int P, int num_special, int grid_w, int head_dim,
                                        double theta, float* rot_out, void* stream) {
   if (frame_idx < 0 || P < 0 || num_special < 0 || num_special > P || grid_w < 1 || head_dim < 6 ||
@@ -893,8 +849,7 @@ namespace {
 swa_status stream_append_pre_impl(swa_stream* h, int global_idx, int frame_idx, const void* x, const float* ln_w,
                                   const float* ln_b, const void* w_qkv, const float* b_qkv, const float* qn_w,
                                   const float* qn_b, const float* kn_w, const float* kn_b, const float* rot,
-                                  float eps, void* xn_ws, void* q_out, void* stream, const RopeGen* gen,
-                                  const void* prep = nullptr) {
+                                  float eps, void* xn_ws, void* q_out, void* stream, const RopeGen* gen) {
   swa_status s = stream_check_layer(h, global_idx);
   if (s != SWA_OK) return s;
   const swa_stream_cfg& c = h->cfg;
@@ -903,15 +858,9 @@ swa_status stream_append_pre_impl(swa_stream* h, int global_idx, int frame_idx, 
   if (!pre_shape_ok(c.P, C, c.heads)) return SWA_ERR_UNSUPPORTED;
   if (!(eps > 0.f)) return SWA_ERR_ARG;
   if (gen && !rope_gen_ok(*gen, c.P)) return SWA_ERR_ARG;
-  if (prep) {
-    const void* ptrs[] = {x, prep, qn_w, qn_b, kn_w, kn_b, q_out};
-    for (const void* q : ptrs)
-      if (!q || !aligned16(q)) return SWA_ERR_ARG;
-  } else {
-    const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, xn_ws, q_out};
-    for (const void* q : ptrs)
-      if (!q || !aligned16(q)) return SWA_ERR_ARG;
-  }
+  const void* ptrs[] = {x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, xn_ws, q_out};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return SWA_ERR_ARG;
   if (!gen && (!rot || !aligned16(rot))) return SWA_ERR_ARG;
   if (frame_idx != h->n_frames[global_idx]) return SWA_ERR_ORDER;
   if (frame_idx >= c.max_frames) return SWA_ERR_CAPACITY;
@@ -929,19 +878,9 @@ swa_status stream_append_pre_impl(swa_stream* h, int global_idx, int frame_idx, 
   uint8_t* kd = layer_k(h, global_idx) + slot_row0 * h->row_bytes;
   uint8_t* vd = layer_v(h, global_idx) + slot_row0 * h->row_bytes;
   return run_attn_pre(x, ln_w, ln_b, w_qkv, b_qkv, qn_w, qn_b, kn_w, kn_b, gen ? nullptr : rot, c.P, C, c.heads,
-                      eps, xn_ws, q_out, kd, vd, st, gen, prep);
+                      eps, xn_ws, q_out, kd, vd, st, gen);
 }
 }  // namespace
-
-extern "C" swa_status swa_stream_append_evict_pre_prepared(swa_stream* h, int global_idx, int frame_idx,
-                                                           const void* x, const void* prep, const float* qn_w,
-                                                           const float* qn_b, const float* kn_w, const float* kn_b,
-                                                           const float* rot, int num_special, int grid_w,
-                                                           double theta, float eps, void* q_out, void* stream) {
-  const RopeGen gen{frame_idx, num_special, grid_w, theta};
-  return stream_append_pre_impl(h, global_idx, frame_idx, x, nullptr, nullptr, nullptr, nullptr, qn_w, qn_b, kn_w,
-                                kn_b, rot, eps, nullptr, q_out, stream, rot ? nullptr : &gen, prep);
-}
 
 extern "C" swa_status swa_stream_append_evict_pre(swa_stream* h, int global_idx, int frame_idx, const void* x,
                                                   const float* ln_w, const float* ln_b, const void* w_qkv,

@@ -179,17 +179,7 @@ struct PreParams {
   // by t, j < rope_nt + rope_nh by h, the rest by w, times rope_inv_freq[j]
   int rope_frame, rope_special, rope_grid_w, rope_nt, rope_nh;
   double rope_inv_freq[64];
-  // norm1 folded into the GEMM (fold_u non-null): A is the raw x, B the prepared
-  // W' = w_qkv diag(ln_w), and the epilogue forms rs * (acc - mu * fold_u[n]) +
-  // fold_v[n] from the token's mean mu and inverse deviation rs, which the
-  // epilogue warps sum from the A tiles as they pass through shared memory
-  const float* fold_u;  // [3C]: column sums of W'
-  const float* fold_v;  // [3C]: ln_b w_qkv^T + b_qkv
 };
-// prepared weights of the folded prologue: W' [3C, C] bf16, then u and v [3C] f32
-size_t attn_pre_weights_bytes(int C);
-cudaError_t launch_attn_pre_prepare(const float* ln_w, const float* ln_b, const void* w_qkv, const float* b_qkv,
-                                    int C, void* prep, cudaStream_t stream);
 cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
                            cudaStream_t stream);
 cudaError_t launch_qkv_pre(const PreParams& p, cudaStream_t stream);

@@ -138,12 +138,10 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
   const uint32_t acc_full = bar0 + 8u * (2 * kPreStages);
   const uint32_t tmem_slot = acc_full + 8;
 
-  const bool fold = p.fold_u != nullptr;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPreStages; ++s) {
       mbar_init(full(s), 1);
-      // folded norm1: the 128 epilogue threads also read each A stage (row sums)
-      mbar_init(empty(s), fold ? 1 + 128 : 1);
+      mbar_init(empty(s), 1);
     }
     mbar_init(acc_full, 1);
     fence_barrier_init();
@@ -203,42 +201,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
     const int quarter = warp & 3;  // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
     const int row = m0 + r;
-    // folded norm1: the token's sum and sum of squares over C, read from row r of
-    // every A stage (64 bf16 in 128 bytes; the 16-byte chunks are visited in a
-    // row-staggered order, which the sum does not see and which spreads a warp's
-    // reads over all banks), each stage released to the producer afterwards
-    float row_mu = 0.f, row_rs = 1.f;
-    bool stats_ok = true;
-    if (fold) {
-      float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-      for (int kc = 0; kc < KC; ++kc) {
-        const int st = kc % kPreStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(full(st), (kc / kPreStages) & 1, p.err, ERR_WAIT_EPI))) {
-          stats_ok = false;
-          break;
-        }
-        const uint32_t rowaddr = base + st * kPreStageBytes + r * 128;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          uint32_t q0, q1, q2, q3;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(q0), "=r"(q1), "=r"(q2), "=r"(q3)
-                       : "r"(rowaddr + (((k + r) & 7) << 4)));
-          const uint32_t qs[4] = {q0, q1, q2, q3};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x2 = make_float2(__uint_as_float(qs[e] << 16), __uint_as_float(qs[e] & 0xffff0000u));
-            s1 = __fadd2_rn(s1, x2);
-            s2 = __ffma2_rn(x2, x2, s2);
-          }
-        }
-        mbar_arrive(empty(st));
-      }
-      const float mu = (s1.x + s1.y) / p.C;
-      row_mu = mu;
-      row_rs = rsqrtf(fmaxf((s2.x + s2.y) / p.C - mu * mu, 0.f) + p.eps);
-    }
-    const bool ok = stats_ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.err, ERR_WAIT_EPI));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.err, ERR_WAIT_EPI));
     if (ok) {
       tc_fence_after();
       const int sec = n0 / p.C;            // 0: q, 1: k, 2: v
@@ -253,21 +216,6 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
         uint32_t a[32];
         tmem_ld32(tmem + lane_off + hh * D + c0, a);
         tmem_wait_ld();
-        if (fold) {
-          // norm1 folded: rs * (x W'^T - mu * u) + v
-          const float* fu = p.fold_u + n0 + hh * D + c0;
-          const float* fv = p.fold_v + n0 + hh * D + c0;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 uu = __ldg(reinterpret_cast<const float4*>(fu + j));
-            const float4 vv = __ldg(reinterpret_cast<const float4*>(fv + j));
-            v[j] = fmaf(row_rs, fmaf(-row_mu, uu.x, __uint_as_float(a[j])), vv.x);
-            v[j + 1] = fmaf(row_rs, fmaf(-row_mu, uu.y, __uint_as_float(a[j + 1])), vv.y);
-            v[j + 2] = fmaf(row_rs, fmaf(-row_mu, uu.z, __uint_as_float(a[j + 2])), vv.z);
-            v[j + 3] = fmaf(row_rs, fmaf(-row_mu, uu.w, __uint_as_float(a[j + 3])), vv.w);
-          }
-          return;
-        }
         const float* bias = p.b_qkv + n0 + hh * D + c0;
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
@@ -421,63 +369,7 @@ cudaError_t launch_pre_d(const PreParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- folded weights
-// One warp per output feature n: W'[n, c] = bf16(w_qkv[n, c] ln_w[c]), u[n] = the
-// sum of W'[n, :] as the GEMM will read it (the rounded bf16 values), v[n] =
-// sum_c ln_b[c] w_qkv[n, c] + b_qkv[n].  Then norm1(x) w_qkv^T + b_qkv equals
-// rs (x W'^T - mu u) + v for a token with mean mu and inverse deviation rs.
-__global__ void __launch_bounds__(256) attn_pre_prepare_kernel(const float* __restrict__ ln_w,
-                                                               const float* __restrict__ ln_b,
-                                                               const __nv_bfloat16* __restrict__ w,
-                                                               const float* __restrict__ b_qkv, int C, int N,
-                                                               __nv_bfloat16* __restrict__ wp, float* __restrict__ u,
-                                                               float* __restrict__ v) {
-  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (n >= N) return;
-  const __nv_bfloat16* wr = w + static_cast<int64_t>(n) * C;
-  __nv_bfloat16* wpr = wp + static_cast<int64_t>(n) * C;
-  float su = 0.f, sv = 0.f;
-  for (int c = lane * 2; c < C; c += 64) {
-    const float w0 = __bfloat162float(wr[c]), w1 = __bfloat162float(wr[c + 1]);
-    const __nv_bfloat16 p0 = __float2bfloat16_rn(w0 * ln_w[c]);
-    const __nv_bfloat16 p1 = __float2bfloat16_rn(w1 * ln_w[c + 1]);
-    wpr[c] = p0;
-    wpr[c + 1] = p1;
-    su += __bfloat162float(p0) + __bfloat162float(p1);
-    sv = fmaf(ln_b[c], w0, fmaf(ln_b[c + 1], w1, sv));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    su += __shfl_xor_sync(0xffffffffu, su, off);
-    sv += __shfl_xor_sync(0xffffffffu, sv, off);
-  }
-  if (lane == 0) {
-    u[n] = su;
-    v[n] = sv + b_qkv[n];
-  }
-}
-
-size_t prep_round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
 }  // namespace
-
-size_t attn_pre_weights_bytes(int C) {
-  const size_t n = 3 * static_cast<size_t>(C);
-  return prep_round256(n * C * 2) + 2 * prep_round256(n * 4);
-}
-
-cudaError_t launch_attn_pre_prepare(const float* ln_w, const float* ln_b, const void* w_qkv, const float* b_qkv,
-                                    int C, void* prep, cudaStream_t stream) {
-  const int N = 3 * C;
-  auto* wp = static_cast<__nv_bfloat16*>(prep);
-  float* u = reinterpret_cast<float*>(static_cast<uint8_t*>(prep) + prep_round256(static_cast<size_t>(N) * C * 2));
-  float* v = u + prep_round256(static_cast<size_t>(N) * 4) / 4;
-  attn_pre_prepare_kernel<<<cdiv(N, 8), 256, 0, stream>>>(ln_w, ln_b, static_cast<const __nv_bfloat16*>(w_qkv),
-                                                           b_qkv, C, N, wp, u, v);
-  count_launches(1);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_ln_rows(const void* x, const float* w, const float* b, void* out, int P, int C, float eps,
                            cudaStream_t stream) {

@@ -219,14 +219,3 @@ def test_binding_argument_counts_match_the_header(swa):
         assert n == len(args), (name, n, len(args))
         checked += 1
     assert checked == len(decls)
-
-
-def test_prepared_prologue_sizes_and_arguments(swa):
-    lib = swa._lib
-    assert lib.swa_attn_pre_weights_bytes(1024) == (3 * 1024 * 1024 * 2) + 2 * ((3 * 1024 * 4 + 255) // 256 * 256)
-    assert lib.swa_attn_pre_weights_bytes(100) == 0 and lib.swa_attn_pre_weights_bytes(4096) == 0
-    assert lib.swa_attn_pre_prepare(None, None, None, None, 1024, None, None) == -1
-    assert lib.swa_attn_pre_prepare(256, 256, 256, 256, 100, 256, None) == -7
-    # generated RoPE asked for with a zero grid width
-    assert lib.swa_attn_pre_prepared(256, 256, 256, 256, 256, 256, None, 0, 5, 0, 1e4, 1004, 1024, 16, 1e-6,
-                                     256, 256, 256, None) == -1

@@ -174,75 +174,3 @@ def test_fused_append_with_generated_rope(swa):
         oc.append_evict(0, i, np.zeros((P, H, D)), np.zeros((P, H, D)))
         assert torch.equal(ks[r0:r0 + P], k_ref) and torch.equal(vs[r0:r0 + P], v_ref)
     assert swa.swa_device_error_check() == 0
-
-
-@pytest.mark.parametrize("P,C,H", [(1004, 1024, 16), (200, 1024, 8), (37, 512, 8)])
-def test_prepared_prologue_matches_oracle(swa, P, C, H):
-    """norm1 folded into the GEMM on prepared weights (W' = w_qkv diag(ln_w), column
-    sums u, bias v): the same q/k/v as the oracle's two-step prologue, within the
-    bf16 tolerance (W' is rounded to bf16 where the two-step path rounds norm1(x))."""
-    inp = synth.prologue_inputs(seed=300 + P + C + H, P=P, C=C, heads=H)
-    d = {k: v.cuda() for k, v in inp.items()}
-    prep = swa.swa_attn_pre_prepare(d["ln_w"], d["ln_b"], d["w_qkv"], d["b_qkv"])
-    q, k, v = swa.swa_attn_pre_prepared(d["x"], prep, d["qn_w"], d["qn_b"], d["kn_w"], d["kn_b"], heads=H,
-                                        rot=d["rot"], eps=EPS)
-    torch.cuda.synchronize()
-    assert swa.swa_device_error_check() == 0
-    rq, rk, rv = _oracle(inp, H)
-    for got, ref, name in ((q, rq, "q"), (k, rk, "k"), (v, rv, "v")):
-        check_bf16(got.float().cpu().numpy(), ref, f"prepared {name} P{P} C{C} H{H}")
-
-
-def test_prepared_weights_are_the_fold(swa):
-    """The prepared blob holds W' = bf16(w_qkv * ln_w), u = row sums of that W',
-    v = ln_b w_qkv^T + b_qkv."""
-    C, H = 512, 8
-    inp = synth.prologue_inputs(seed=5, P=16, C=C, heads=H)
-    d = {k: v.cuda() for k, v in inp.items()}
-    prep = swa.swa_attn_pre_prepare(d["ln_w"], d["ln_b"], d["w_qkv"], d["b_qkv"]).cpu()
-    nw = 3 * C * C * 2
-    wp = prep[:nw].view(torch.bfloat16).view(3 * C, C)
-    off = (nw + 255) // 256 * 256
-    u = prep[off:off + 3 * C * 4].view(torch.float32)
-    off2 = off + (3 * C * 4 + 255) // 256 * 256
-    v = prep[off2:off2 + 3 * C * 4].view(torch.float32)
-    w = inp["w_qkv"].float()
-    assert torch.equal(wp, (w * inp["ln_w"][None, :]).to(torch.bfloat16))
-    np.testing.assert_allclose(u.numpy(), wp.double().sum(1).numpy(), rtol=1e-5, atol=1e-4)
-    want_v = (inp["ln_b"].double()[None, :] * w.double()).sum(1) + inp["b_qkv"].double()
-    np.testing.assert_allclose(v.numpy(), want_v.numpy(), rtol=1e-5, atol=1e-5)
-
-
-def test_prepared_prologue_generated_rope_and_stream_append(swa):
-    """Generated 3-D RoPE on prepared weights against the oracle at frame 999, and
-    the streaming append on prepared weights writing exactly that K/V into the slot."""
-    P, C, H, S, Wc, F = 5 + 37 * 27, 1024, 16, 1, 2, 3
-    D = C // H
-    inp = synth.prologue_inputs(seed=41, P=P, C=C, heads=H)
-    d = {k: v.cuda() for k, v in inp.items()}
-    prep = swa.swa_attn_pre_prepare(d["ln_w"], d["ln_b"], d["w_qkv"], d["b_qkv"])
-    q, k, v = swa.swa_attn_pre_prepared(d["x"], prep, d["qn_w"], d["qn_b"], d["kn_w"], d["kn_b"], heads=H,
-                                        frame_idx=999, num_special=5, grid_w=27, eps=EPS)
-    torch.cuda.synchronize()
-    a = {n: t.double().numpy() for n, t in inp.items()}
-    a["rot"] = orc.rope3d_table(999, P, 5, 27, D)
-    rq, rk, rv = orc.attn_pre(a["x"], *(a[n] for n in ORDER), heads=H, eps=EPS)
-    for got, ref, name in ((q, rq, "q"), (k, rk, "k"), (v, rv, "v")):
-        check_bf16(got.float().cpu().numpy(), ref, f"prepared {name}, generated RoPE")
-    cache = swa.SwaStream(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, max_frames=F,
-                          dtype=torch.bfloat16)
-    ks, vs = cache.storage(0, "k"), cache.storage(0, "v")
-    ppf = -(-P // 16)
-    oc = orc.StreamCache(heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, page_tokens=16, max_frames=F)
-    for i in range(F):
-        qi, ki, vi = swa.swa_attn_pre_prepared(d["x"], prep, d["qn_w"], d["qn_b"], d["kn_w"], d["kn_b"], heads=H,
-                                               frame_idx=i, num_special=5, grid_w=27, eps=EPS)
-        q_out = torch.empty_like(qi)
-        cache.swa_stream_append_evict_pre_prepared(0, i, d["x"], prep, d["qn_w"], d["qn_b"], d["kn_w"], d["kn_b"],
-                                                   q_out, num_special=5, grid_w=27, eps=EPS)
-        torch.cuda.synchronize()
-        assert torch.equal(q_out, qi)
-        r0 = oc.slot_of(i) * ppf * 16
-        oc.append_evict(0, i, np.zeros((P, H, D)), np.zeros((P, H, D)))
-        assert torch.equal(ks[r0:r0 + P], ki) and torch.equal(vs[r0:r0 + P], vi)
-    assert swa.swa_device_error_check() == 0
