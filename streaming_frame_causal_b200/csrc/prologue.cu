@@ -49,12 +49,21 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
   constexpr int kMaxChunks = 8;  // C <= 2048
   const int nch = C / 256;       // 8-element chunks per lane
   const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * C;
-  // all of the row's loads are issued before any is used (no early exit in the
-  // loop, so the unrolled loads are independent)
+  // all of the row's loads, the LayerNorm weight and bias included, are issued
+  // before any is used (no early exit in the loop, so the unrolled loads are
+  // independent): one memory round trip per row
   uint4 raw[kMaxChunks];
+  float4 wq[kMaxChunks][2], bq[kMaxChunks][2];
 #pragma unroll
-  for (int c = 0; c < kMaxChunks; ++c)
-    raw[c] = (c < nch) ? *reinterpret_cast<const uint4*>(xr + (c * 32 + lane) * 8) : make_uint4(0, 0, 0, 0);
+  for (int c = 0; c < kMaxChunks; ++c) {
+    const int col = (c * 32 + lane) * 8;
+    const bool in = c < nch;
+    raw[c] = in ? *reinterpret_cast<const uint4*>(xr + col) : make_uint4(0, 0, 0, 0);
+    wq[c][0] = in ? __ldg(reinterpret_cast<const float4*>(w + col)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wq[c][1] = in ? __ldg(reinterpret_cast<const float4*>(w + col + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bq[c][0] = in ? __ldg(reinterpret_cast<const float4*>(b + col)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bq[c][1] = in ? __ldg(reinterpret_cast<const float4*>(b + col + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float v[kMaxChunks * 8];
   float s = 0.f;
 #pragma unroll
@@ -90,10 +99,7 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __res
   for (int c = 0; c < kMaxChunks; ++c) {
     if (c >= nch) break;
     const int col = (c * 32 + lane) * 8;
-    const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + col));
-    const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + col + 4));
-    const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + col));
-    const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + col + 4));
+    const float4 w0 = wq[c][0], w1 = wq[c][1], b0 = bq[c][0], b1 = bq[c][1];
     const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
     const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     uint32_t o[4];
@@ -120,7 +126,10 @@ constexpr int kPreABytes = kPreM * 64 * 2;  // 16 KB: 128 rows x 64 columns
 constexpr int kPreBBytes = kPreN * 64 * 2;  // 16 KB
 constexpr int kPreStageBytes = kPreABytes + kPreBBytes;
 constexpr int kPreOffBar = kPreStages * kPreStageBytes;
-constexpr int kPreSmem = kPreOffBar + (2 * kPreStages + 1) * 8 + 16 + 1024;
+// the tile's per-feature epilogue constants, staged once: bias, then the q/k
+// norm weight and bias of each feature's head position (3 x 128 floats)
+constexpr int kPreOffPar = kPreOffBar + 128;
+constexpr int kPreSmem = kPreOffPar + 3 * kPreN * 4 + 1024;
 
 template <int D>
 __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_constant__ PreParams p) {
@@ -201,14 +210,32 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
     const int quarter = warp & 3;  // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
     const int row = m0 + r;
+    const int sec = n0 / p.C;            // 0: q, 1: k, 2: v
+    const int h0 = (n0 - sec * p.C) / D;  // first head of this tile
+    // while the main loop runs, stage the tile's bias and norm constants in
+    // shared memory (thread r takes feature r of the tile), so the epilogue's
+    // loop reads no global memory except the RoPE table
+    float* par = reinterpret_cast<float*>(gbase + kPreOffPar);
+    {
+      const float* nwg = sec == 0 ? p.qn_w : p.kn_w;
+      const float* nbg = sec == 0 ? p.qn_b : p.kn_b;
+      par[r] = __ldg(p.b_qkv + n0 + r);
+      par[kPreN + r] = sec < 2 ? __ldg(nwg + (r % D)) : 0.f;
+      par[2 * kPreN + r] = sec < 2 ? __ldg(nbg + (r % D)) : 0.f;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+    // head_dim 64: this token's RoPE table row (32 pairs, the same for both
+    // heads of the tile) is loaded into registers before the accumulator is ready
+    float4 rotv[D == 64 ? 16 : 1];
+    if constexpr (D == 64) {
+      const float4* rt = reinterpret_cast<const float4*>(p.rot + static_cast<int64_t>(row < p.P ? row : 0) * D);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) rotv[i] = (p.rot && row < p.P) ? __ldg(rt + i) : make_float4(1.f, 0.f, 1.f, 0.f);
+    }
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, p.err, ERR_WAIT_EPI));
     if (ok) {
       tc_fence_after();
-      const int sec = n0 / p.C;            // 0: q, 1: k, 2: v
-      const int h0 = (n0 - sec * p.C) / D;  // first head of this tile
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-      const float* nw = sec == 0 ? p.qn_w : p.kn_w;
-      const float* nb = sec == 0 ? p.qn_b : p.kn_b;
 
       // load 32 columns of this thread's row (+ bias) from TMEM
       auto load32 = [&](int hh, int c0, float* v) {
@@ -216,10 +243,10 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
         uint32_t a[32];
         tmem_ld32(tmem + lane_off + hh * D + c0, a);
         tmem_wait_ld();
-        const float* bias = p.b_qkv + n0 + hh * D + c0;
+        const float4* bias = reinterpret_cast<const float4*>(par + hh * D + c0);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-          const float4 bb = __ldg(reinterpret_cast<const float4*>(bias + j));
+          const float4 bb = bias[j / 4];
           v[j] = __uint_as_float(a[j]) + bb.x;
           v[j + 1] = __uint_as_float(a[j + 1]) + bb.y;
           v[j + 2] = __uint_as_float(a[j + 2]) + bb.z;
@@ -256,15 +283,15 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
           mean = s1 / D;
           rs = rsqrtf(fmaxf(s2 / D - mean * mean, 0.f) + p.eps);
         }
-#pragma unroll 1
+#pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           float v[32];
           load32(hh, c0, v);
           if (sec < 2) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-              const float4 ww = __ldg(reinterpret_cast<const float4*>(nw + c0 + j));
-              const float4 bb = __ldg(reinterpret_cast<const float4*>(nb + c0 + j));
+              const float4 ww = *reinterpret_cast<const float4*>(par + kPreN + hh * D + c0 + j);
+              const float4 bb = *reinterpret_cast<const float4*>(par + 2 * kPreN + hh * D + c0 + j);
               v[j] = (v[j] - mean) * rs * ww.x + bb.x;
               v[j + 1] = (v[j + 1] - mean) * rs * ww.y + bb.y;
               v[j + 2] = (v[j + 2] - mean) * rs * ww.z + bb.z;
@@ -275,7 +302,7 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
               const float4* rt = reinterpret_cast<const float4*>(p.rot + static_cast<int64_t>(row) * D + c0);
 #pragma unroll
               for (int j = 0; j < 32; j += 4) {
-                const float4 cs = __ldg(rt + j / 4);
+                const float4 cs = (D == 64) ? rotv[((c0 + j) / 4) % (D == 64 ? 16 : 1)] : __ldg(rt + j / 4);
                 const float x0 = v[j], x1 = v[j + 1], x2 = v[j + 2], x3 = v[j + 3];
                 v[j] = x0 * cs.x - x1 * cs.y;
                 v[j + 1] = x0 * cs.y + x1 * cs.x;
