@@ -195,8 +195,11 @@ swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx,
 /* The frame's queries q_frame [P, heads, head_dim] attend to everything the layer's
  * cache holds after the append (retained full frames, the current frame and
  * retained specials); out [P, heads, head_dim].  ``frame_idx`` must be the frame
- * appended last (SWA_ERR_ORDER otherwise).  Uses split-KV partials in the handle's
- * buffer: calls on one handle must not overlap on the GPU. */
+ * appended last (SWA_ERR_ORDER otherwise).  The keys are split across CTAs; each
+ * writes its partial (O, max, sum) into the handle's buffer and the last CTA of
+ * each (head, query-tile pair) to finish merges them into ``out`` (one launch, an
+ * arrival counter per pair in the handle's buffer): calls on one handle must not
+ * overlap on the GPU. */
 swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx,
                              const void* q_frame, void* out, void* stream);
 
@@ -373,7 +376,7 @@ swa_status swa_band_prefill(const void* q, const void* k, const void* v, void* o
  *   k_cache, v_cache: [B, W, Hkv, head_dim] (updated in place).
  *   workspace: device scratch of at least swa_decode_workspace_bytes(...) bytes
  *   (split-K partials); calls sharing a workspace must not overlap on the GPU.
- * bf16: head_dim 64 or 128 with Hq/Hkv in {1, 2, 4, 8} (other group sizes return
+ * bf16: head_dim 64 or 128 with Hq/Hkv from 1 to 8 (larger groups return
  * SWA_ERR_UNSUPPORTED); f32: head_dim 32, 64 or 128, any Hq/Hkv.  The kernels read
  * only the valid slots' values: slots beyond ``pos`` may hold anything, NaN
  * included. */
@@ -392,7 +395,7 @@ swa_status swa_decode(const void* q, const void* k_new, const void* v_new,
  * offers no way to obtain memory.
  *
  * swa_decode_noalloc does what swa_decode does for bf16 (head_dim 64 or 128,
- * Hq/Hkv in {1,2,4,8}) with the same arguments minus the workspace: its split-K
+ * Hq/Hkv from 1 to 8) with the same arguments minus the workspace: its split-K
  * scratch is a fixed SWA_DECODE_NOALLOC_SCRATCH_BYTES array inside the library,
  * held on every GPU that loads the library until the process exits.  It calls no
  * allocating routine.  Requests whose scratch would exceed the array return

@@ -475,7 +475,7 @@ extern "C" swa_status swa_decode(const void* q, const void* k_new, const void* v
   }
   if (head_dim != 64 && head_dim != 128) return SWA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return SWA_ERR_UNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, Hq, Hkv, head_dim, W);
   if (!workspace || workspace_bytes < need) return SWA_ERR_CAPACITY;
   if (!aligned16(workspace)) return SWA_ERR_ARG;

@@ -236,15 +236,14 @@ SWA_DEV Work decode_work(const TcParams& p) {
 
 // How the 64 exponential pairs of a 128-column row are split (per group of 8 pairs):
 // the first kPolyPairs take 2^x on the FMA pipe (polynomial), the rest two f32
-// MUFU exp2 (packed f16x2/bf16x2 MUFU exp2 yields no more results per clock).
-// Measured on B200 (same-box sweeps of 2, 3, 4): 3 is fastest at head_dim 64,
-// where the row sums come from the tensor core and leave the FMA pipe room, and
-// 2 at head_dim 128.  SWA_POLY_PAIRS_D64 / _D128 override them for tuning builds.
+// MUFU exp2.  Measured on B200 with the warp issuer (same-box A/B): at head_dim
+// 64, 3 beats 2 and 4 by 1-8 %; at head_dim 128, 1 beats 0 and 2 by 2-5 %.
+// SWA_POLY_PAIRS_D64 / _D128 override them for tuning builds.
 #ifndef SWA_POLY_PAIRS_D64
 #define SWA_POLY_PAIRS_D64 3
 #endif
 #ifndef SWA_POLY_PAIRS_D128
-#define SWA_POLY_PAIRS_D128 2
+#define SWA_POLY_PAIRS_D128 1
 #endif
 template <int D>
 constexpr int kPolyPairs = (D == 64) ? SWA_POLY_PAIRS_D64 : SWA_POLY_PAIRS_D128;

@@ -66,7 +66,7 @@ extern "C" swa_status swa_decode_noalloc(const void* q, const void* k_new, const
   // only the bf16 decode uses scratch memory; the f32 decode needs none (use swa_decode)
   if (dtype != SWA_BF16 || (head_dim != 64 && head_dim != 128)) return SWA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return SWA_ERR_UNSUPPORTED;
   if (B == 0) return SWA_OK;
   // reject requests whose partials do not fit the fixed array
   const size_t need = swa::decode_workspace_bytes(B, Hq, Hkv, head_dim, W);

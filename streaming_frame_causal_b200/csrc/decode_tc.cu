@@ -524,9 +524,7 @@ DecodeTcPlan decode_tc_plan(int B, int Hkv, int n_valid, int max_pieces, int sms
   return pl;
 }
 
-bool decode_tc_supported(int D, int G) {
-  return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
-}
+bool decode_tc_supported(int D, int G) { return (D == 64 || D == 128) && G >= 1 && G <= 8; }
 
 // p.chunks on entry: the partial slots the workspace holds per (batch, KV head)
 cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t stream) {
@@ -549,14 +547,22 @@ cudaError_t launch_decode_tc(const DecodeParams& p_in, int sms, cudaStream_t str
     switch (G) {
       case 1: e = launch_tcd<128, 1>(p, grid, stream); break;
       case 2: e = launch_tcd<128, 2>(p, grid, stream); break;
+      case 3: e = launch_tcd<128, 3>(p, grid, stream); break;
       case 4: e = launch_tcd<128, 4>(p, grid, stream); break;
+      case 5: e = launch_tcd<128, 5>(p, grid, stream); break;
+      case 6: e = launch_tcd<128, 6>(p, grid, stream); break;
+      case 7: e = launch_tcd<128, 7>(p, grid, stream); break;
       default: e = launch_tcd<128, 8>(p, grid, stream); break;
     }
   } else {
     switch (G) {
       case 1: e = launch_tcd<64, 1>(p, grid, stream); break;
       case 2: e = launch_tcd<64, 2>(p, grid, stream); break;
+      case 3: e = launch_tcd<64, 3>(p, grid, stream); break;
       case 4: e = launch_tcd<64, 4>(p, grid, stream); break;
+      case 5: e = launch_tcd<64, 5>(p, grid, stream); break;
+      case 6: e = launch_tcd<64, 6>(p, grid, stream); break;
+      case 7: e = launch_tcd<64, 7>(p, grid, stream); break;
       default: e = launch_tcd<64, 8>(p, grid, stream); break;
     }
   }

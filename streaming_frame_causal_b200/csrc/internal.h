@@ -137,7 +137,7 @@ struct DecodeParams {
 };
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W);
-// tensor-core decode (head_dim 128, G in {1, 2, 4, 8}): appends the new token,
+// tensor-core decode (head_dim 64 or 128, G = 1..8): appends the new token,
 // runs the persistent kernel and the combine; p.chunks = partial slots available
 bool decode_tc_supported(int D, int G);
 int decode_tc_pieces(int B, int Hkv, int n_valid, int max_pieces, int sms);

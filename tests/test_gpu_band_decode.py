@@ -54,6 +54,11 @@ def test_band_parity(swa, N, Hq, Hkv, D, W, dtype):
     # head_dim 64 on the same kernel (one 64-column sub-tile per key tile)
     (2, 700, 699, 8, 4, 64, torch.bfloat16),
     (3, 300, 1000, 8, 8, 64, torch.bfloat16),
+    # group sizes that are not powers of two: 3, 5, 6 and 7 query heads per KV head
+    (2, 512, 2000, 12, 4, 128, torch.bfloat16),
+    (2, 260, 259, 10, 2, 64, torch.bfloat16),
+    (1, 384, 5000, 24, 4, 128, torch.bfloat16),
+    (2, 200, 150, 14, 2, 64, torch.bfloat16),
 ])
 def test_decode_parity(swa, B, W, pos, Hq, Hkv, D, dtype):
     q, kn, vn, kc, vc = synth.decode_inputs(seed=pos, B=B, W=W, Hq=Hq, Hkv=Hkv, D=D, dtype=dtype)
