@@ -108,7 +108,7 @@ struct Plan {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffOnes = kOffV + kStages * kTileBytes;  // the constant block (kSumCol)
   static constexpr int kOffBar = kOffOnes + (kSumCol ? kSubBytes : 0);
-  static constexpr int kNumBars = 2 + 4 * kStages + 3 + 2 + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 + 4 * kStages + 3 + 2 + 2 + 2 + 2 + 2;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;   // TMEM base (4 bytes), then the merge flag
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
 };
@@ -281,7 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   auto v_empty = [&](int s) { return bar0 + 8u * (2 + 3 * PL::kStages + s); };
   constexpr int kB = 2 + 4 * PL::kStages;
   auto s_full = [&](int i) { return bar0 + 8u * (kB + i); };      // per S buffer (3 in the ring)
-  auto p_full = [&](int g) { return bar0 + 8u * (kB + 3 + g); };
+  // P hand-off j of query tile g (128 arrivals, one per row) goes to barrier j mod 2, and
+  // the issuer waits for it with parity (j / 2) mod 2.  One barrier per tile would not do:
+  // the S of key tile j + 1 can be ready before every warp of the tile has handed off P_j
+  // (the ring computes it early), so a warp running a whole key tile ahead of a slower one
+  // would arrive for j + 1 while the other is still on j, and its arrivals would complete
+  // hand-off j without the slower warp's rows of P
+  auto p_full = [&](int g, int j) { return bar0 + 8u * ((j & 1) ? kB + 11 + g : kB + 3 + g); };
+  auto p_parity = [](int j) { return static_cast<uint32_t>((j >> 1) & 1); };
   auto o_full = [&](int g) { return bar0 + 8u * (kB + 5 + g); };
   auto drain = [&](int g) { return bar0 + 8u * (kB + 7 + g); };
   auto o_done = [&](int g) { return bar0 + 8u * (kB + 9 + g); };  // ring: PV_g(j) complete
@@ -301,8 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     mbar_init(s_full(2), 1);
     mbar_init(o_done(0), 1);
     mbar_init(o_done(1), 1);
-    mbar_init(p_full(0), 128);
-    mbar_init(p_full(1), 128);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(p_full(g, 0), 128);
+      mbar_init(p_full(g, 1), 128);
+    }
     for (int g = 0; g < 2; ++g) {
       mbar_init(o_full(g), 1);
       mbar_init(drain(g), 1);
@@ -477,12 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
         for (int j = 0; j < T && ok; ++j) {
-          if (!wait(p_full(0), j & 1)) break;
+          if (!wait(p_full(0, j), p_parity(j))) break;
           tc_fence_after();
           pv_ring(0, j);
           if (has_b) {
             if (j + 1 < T) qk_ring(1, j + 1);
-            if (!wait(p_full(1), j & 1)) break;
+            if (!wait(p_full(1, j), p_parity(j))) break;
             tc_fence_after();
             pv_ring(1, j);
           }
@@ -517,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (PL::kSplitKV && !wait(v_full(st), (j / PL::kStages) & 1)) break;
 #pragma unroll 1
         for (int g = 0; g < ng; ++g) {
-          if (!wait(p_full(g), j & 1)) {
+          if (!wait(p_full(g, j), p_parity(j))) {
             ok = false;
             break;
           }
@@ -606,9 +615,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
       } else if (kvalid < kRows) {
+        // only the 32-column blocks that reach past the run's end (kvalid is
+        // the same for every row, so the block test is warp-uniform)
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= kvalid) s[c] = __float_as_uint(-INFINITY);
+        for (int c0 = 0; c0 < 128; c0 += 32)
+          if (kvalid < c0 + 32) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c0 + c >= kvalid) s[c0 + c] = __float_as_uint(-INFINITY);
+          }
       }
       // ---- row max: eight independent 3-input max chains
       float a[8];
@@ -692,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tmem_st32(tP + 32, s + 32);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(g));
+      mbar_arrive(p_full(g, j));
     }
     // ---- epilogue
     if (active && ok) {
@@ -771,8 +786,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const int64_t stride = static_cast<int64_t>(p.Nq) * p.Hq;
           const int64_t base_idx = static_cast<int64_t>(row) * p.Hq + my_h;
           float M = -INFINITY;
+#pragma unroll 4
           for (int c = 0; c < p.splits; ++c) M = fmaxf(M, __ldcg(p.part_ml + (c * stride + base_idx) * 2));
           float L = 0.f;
+#pragma unroll 4
           for (int c = 0; c < p.splits; ++c) {
             const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (c * stride + base_idx) * 2));
             L = fmaf((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M), ml.y, L);
@@ -782,11 +799,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * out_ld +
                                static_cast<int64_t>(p.out_h0 + my_h) * D;
           // 32 output columns at a time, each the weighted sum over the splits
+          // (four splits' loads in flight at once)
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             float o[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0.f;
+#pragma unroll 4
             for (int c = 0; c < p.splits; ++c) {
               const float m_c = __ldcg(p.part_ml + (c * stride + base_idx) * 2);
               const float wc = (m_c == -INFINITY) ? 0.f : exp2f(m_c - M);
