@@ -26,6 +26,7 @@ constexpr int kDecRows = 32;
 // merge the per-piece partials: one warp per (batch, query head)
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeParams p) {
+  griddep_wait();  // launched behind the decode (programmatic launch): its partials first
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq) return;
@@ -102,17 +103,14 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int W) {
 }
 
 cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t stream) {
-  if (p.D == 128)
-    decode_combine_kernel<128><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
-  else if (p.D == 64)
-    decode_combine_kernel<64><<<(p.B * p.Hq + 7) / 8, 256, 0, stream>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  const dim3 grid((p.B * p.Hq + 7) / 8);
+  if (p.D == 128) return launch_after(decode_combine_kernel<128>, grid, dim3(256), 0, stream, p);
+  if (p.D == 64) return launch_after(decode_combine_kernel<64>, grid, dim3(256), 0, stream, p);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t stream) {
-  // head_dim 64 and 128, 1, 2, 4 or 8 query heads per KV head: the tensor-core
+  // head_dim 64 and 128, 1 to 8 query heads per KV head: the tensor-core
   // kernel (decode_tc.cu); the entry points accept no other bf16 shape
   if (!decode_tc_supported(p.D, p.Hq / p.Hkv)) return cudaErrorInvalidValue;
   return launch_decode_tc(p, device_sms(), stream);

@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_units = p.B * p.Hkv * p.chunks;
+  griddep_launch_dependents();  // the combine launches now and waits for this grid
 
   const uint32_t bar0 = base + kOffBar;
   auto q_full = [&](int i) { return bar0 + 8u * i; };
@@ -189,6 +190,9 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
         for (int sub = 0; sub < PL::kSubs; ++sub)
           tma_load_2d(base + kOffQ + qb * kTcdSmall + sub * kTcdSmallSub, &p.tm_q, q_full(qb), sub * 64,
                       u.b * p.Hq + u.kvh * G);
+        // the new token's append (the kernel ahead, programmatic launch) must have
+        // landed before the first cache tile is read; Q is an input of its own
+        if (lu == 0) griddep_wait();
         ++lu;
         for (int j = 0; j < u.T; ++j, ++jj) {
           const int st = jj % kTcdStages;
@@ -466,6 +470,7 @@ __global__ void __launch_bounds__(kTcdThreads, 1) decode_tc_kernel(const __grid_
 
 // the new token's K/V into slot pos mod W of every (batch, KV head), 16 bytes a thread
 __global__ void decode_append_kernel(const DecodeParams p) {
+  griddep_launch_dependents();  // the decode sets up and loads Q meanwhile
   const int64_t per_b = static_cast<int64_t>(p.Hkv) * p.D / 8;  // 16-byte chunks of one token
   const int64_t n = static_cast<int64_t>(p.B) * per_b;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -489,8 +494,8 @@ cudaError_t launch_tcd(const DecodeParams& p, int grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set.mark(dev);
   }
-  decode_tc_kernel<D, G><<<grid, kTcdThreads, kSmem, stream>>>(p);
-  return cudaGetLastError();
+  // after the append on the same stream: programmatic launch (see the producer)
+  return launch_after(decode_tc_kernel<D, G>, dim3(grid), dim3(kTcdThreads), kSmem, stream, p);
 }
 
 }  // namespace

@@ -197,6 +197,26 @@ int* device_error_flag();
 int device_ready_status(int** err);
 // counts kernel launches (every launch_* helper adds what it enqueued)
 void count_launches(int n);
+
+// Launch ``kernel`` so that it may start before the kernel ahead of it on
+// ``stream`` has finished (programmatic dependent launch): the kernel's own set-up
+// and its loads of inputs that kernel does not write overlap that kernel's tail;
+// it calls griddep_wait() before touching anything the kernel ahead writes.
+template <typename... Params, typename... Args>
+cudaError_t launch_after(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_debug_wait(int* err, long long timeout_ns, cudaStream_t stream);
 

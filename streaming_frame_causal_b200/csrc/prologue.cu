@@ -43,6 +43,7 @@ SWA_DEV void tma_load_2d(uint32_t dst, const void* tmap, uint32_t mbar, int c0, 
 __global__ void __launch_bounds__(256) ln_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                       const float* __restrict__ w, const float* __restrict__ b,
                                                       __nv_bfloat16* __restrict__ out, int P, int C, float eps) {
+  griddep_launch_dependents();  // the qkv GEMM may set up and load weights meanwhile
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= P) return;
@@ -168,10 +169,19 @@ __global__ void __launch_bounds__(kPreThreads, 2) qkv_pre_kernel(const __grid_co
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_a);
       tma_prefetch_desc(&p.tm_b);
-      int issued = 0;
-      for (int kc = 0; kc < KC; ++kc) {
+      // the first stages' weight tiles do not depend on norm1, which may still
+      // run (programmatic launch): load them, then wait for norm1's output
+      const int first = KC < kPreStages ? KC : kPreStages;
+      for (int kc = 0; kc < first; ++kc) {
+        mbar_arrive_expect_tx(full(kc), kPreStageBytes);
+        tma_load_2d(base + kc * kPreStageBytes + kPreABytes, &p.tm_b, full(kc), kc * 64, n0);
+      }
+      griddep_wait();
+      for (int kc = 0; kc < first; ++kc) tma_load_2d(base + kc * kPreStageBytes, &p.tm_a, full(kc), kc * 64, m0);
+      int issued = first;
+      for (int kc = first; kc < KC; ++kc) {
         const int s = kc % kPreStages;
-        if (kc >= kPreStages && !mbar_wait(empty(s), ((kc / kPreStages) - 1) & 1, p.err, ERR_WAIT_TMA)) break;
+        if (!mbar_wait(empty(s), ((kc / kPreStages) - 1) & 1, p.err, ERR_WAIT_TMA)) break;
         const uint32_t dst = base + s * kPreStageBytes;
         mbar_arrive_expect_tx(full(s), kPreStageBytes);
         tma_load_2d(dst, &p.tm_a, full(s), kc * 64, m0);
@@ -391,9 +401,10 @@ cudaError_t launch_pre_d(const PreParams& p, cudaStream_t stream) {
     attr_set.mark(dev);
   }
   dim3 grid(cdiv(p.P, kPreM), 3 * p.C / kPreN);
-  qkv_pre_kernel<D><<<grid, kPreThreads, kPreSmem, stream>>>(p);
+  // after norm1 on the same stream: programmatic launch (see the producer)
+  const cudaError_t e = launch_after(qkv_pre_kernel<D>, grid, dim3(kPreThreads), kPreSmem, stream, p);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace

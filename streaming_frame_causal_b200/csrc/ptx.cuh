@@ -39,6 +39,15 @@ SWA_DEV void mbar_init(uint32_t addr, uint32_t count) {
 // proxy (the tensor core and TMA)
 SWA_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute (launch_after in internal.h) may start while
+// the kernel ahead of it on the stream still runs.  griddep_wait() returns once
+// that kernel has completed and its memory is visible; griddep_launch_dependents()
+// lets the kernel behind this one start launching once every CTA of this grid has
+// signalled or exited.  Without such a launch both return at once.
+SWA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SWA_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 SWA_DEV void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
