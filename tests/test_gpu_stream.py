@@ -263,3 +263,45 @@ def test_no_scale_frames(swa):
             frames_to_check=set(range(10)))
     _stream(swa, F=10, P=300, H=2, D=64, S=0, Wc=3, special=True, dtype=torch.bfloat16,
             frames_to_check={3, 6, 9})
+
+
+def test_split_attend_equals_one_split_over_a_long_stream(swa):
+    """Full size (8 scale + 64 window frames of 1004 tokens, 16 x 64), 30
+    keyframe attends in steady state and two non-keyframes, each through a cache
+    whose attend is split into pieces (partials merged by the CTA that finishes
+    an item last) and through one that runs every item whole: every (query row,
+    head) agrees within bf16 rounding, so no piece's partial is lost, merged
+    twice or read before it was written (a block of 32 rows from one softmax warp
+    is the failure this looks for)."""
+    P, H, D, S, Wc = 1004, 16, 64, 8, 64
+    kw = dict(num_layers=1, heads=H, head_dim=D, P=P, scale_frames=S, window_frames=Wc, max_frames=120,
+              dtype=torch.bfloat16)
+    split, whole = swa.SwaStream(max_splits=12, **kw), swa.SwaStream(max_splits=1, **kw)
+    frames = [tuple(t.cuda() for t in synth.stream_frame(i, P=P, H=H, D=D)) for i in range(8)]
+    extra = tuple(t.cuda() for t in synth.stream_frame(5_000, P=P, H=H, D=D, base_seed=3))
+
+    def agree(a, b, what):
+        a, b = a.float(), b.float()
+        assert torch.isfinite(a).all(), what
+        num = (a - b).norm(dim=2)
+        den = b.norm(dim=2).clamp_min(1e-6)
+        worst = float((num / den).max())
+        assert worst <= 2e-2, f"{what}: worst (row, head) relative error {worst:.3e}"
+
+    for i in range(100):
+        q, k, v = frames[i % 8]
+        if i in (80, 95):
+            oa = torch.full((P, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+            ob = torch.full_like(oa, float("nan"))
+            split.swa_stream_attend_transient(0, *extra, oa)
+            whole.swa_stream_attend_transient(0, *extra, ob)
+            agree(oa, ob, f"non-keyframe before keyframe {i}")
+        split.swa_stream_append_evict(0, i, k, v)
+        whole.swa_stream_append_evict(0, i, k, v)
+        if i >= 70:
+            oa = torch.full((P, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+            ob = torch.full_like(oa, float("nan"))
+            split.swa_stream_attend(0, i, q, oa)
+            whole.swa_stream_attend(0, i, q, ob)
+            agree(oa, ob, f"keyframe {i}")
+    assert swa.swa_device_error_check() == 0
