@@ -195,11 +195,11 @@ swa_status swa_stream_append_evict(swa_stream* h, int global_idx, int frame_idx,
 /* The frame's queries q_frame [P, heads, head_dim] attend to everything the layer's
  * cache holds after the append (retained full frames, the current frame and
  * retained specials); out [P, heads, head_dim].  ``frame_idx`` must be the frame
- * appended last (SWA_ERR_ORDER otherwise).  The keys are split across CTAs; each
- * writes its partial (O, max, sum) into the handle's buffer and the last CTA of
- * each (head, query-tile pair) to finish merges them into ``out`` (one launch, an
- * arrival counter per pair in the handle's buffer): calls on one handle must not
- * overlap on the GPU. */
+ * appended last (SWA_ERR_ORDER otherwise).  The keys are split across CTAs (at
+ * most cfg.max_splits per query tile); each writes its partial (O, max, sum) into
+ * the handle's buffer and a combine kernel, launched behind the attend on the same
+ * stream, merges them into ``out`` (two launches; one when a frame needs a single
+ * split): calls on one handle must not overlap on the GPU. */
 swa_status swa_stream_attend(swa_stream* h, int global_idx, int frame_idx,
                              const void* q_frame, void* out, void* stream);
 

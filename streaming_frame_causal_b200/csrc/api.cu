@@ -501,7 +501,6 @@ struct swa_stream {
   uint8_t* store0;
   float* part_o;
   float* part_ml;
-  int* split_cnt;  // per attend work item: CTAs of the item that have written their partials
   std::vector<int> n_frames;
   std::vector<CUtensorMap> tm_k, tm_v;
 };
@@ -544,11 +543,9 @@ bool stream_geom(const swa_stream_cfg* c, StreamGeom* g) {
   g->meta_stride = round256(static_cast<size_t>(g->meta_ints + 8 + 2 * (g->max_segs + 1)) * 4);
   g->store_bytes = round256(static_cast<size_t>(g->total_rows) * g->row_bytes);
   const size_t rows_h = static_cast<size_t>(c->P) * c->heads;
-  // split-KV partials (O, then max and sum), then one arrival counter per attend
-  // work item (head x query-tile pair) for the merge in the attend's last CTA
+  // split-KV partials of the attend: O, then max and sum
   g->part_bytes = round256(static_cast<size_t>(c->max_splits) * rows_h * c->head_dim * 4) +
-                  round256(static_cast<size_t>(c->max_splits) * rows_h * 2 * 4) +
-                  round256(static_cast<size_t>(c->heads) * qpairs_per_frame(c->P) * 4);
+                  round256(static_cast<size_t>(c->max_splits) * rows_h * 2 * 4);
   g->total = g->meta_stride * c->num_layers + 2 * g->store_bytes * c->num_layers + g->part_bytes;
   return true;
 }
@@ -612,8 +609,6 @@ extern "C" swa_status swa_stream_init(swa_stream** out, const swa_stream_cfg* cf
   h->part_o = reinterpret_cast<float*>(part);
   h->part_ml = reinterpret_cast<float*>(part + round256(static_cast<size_t>(cfg->max_splits) * rows_h *
                                                         cfg->head_dim * 4));
-  h->split_cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(h->part_ml) +
-                                        round256(static_cast<size_t>(cfg->max_splits) * rows_h * 2 * 4));
   h->n_frames.assign(cfg->num_layers, 0);
   if (cfg->dtype == SWA_BF16) {
     h->tm_k.resize(cfg->num_layers);
@@ -645,8 +640,6 @@ extern "C" swa_status swa_stream_reset(swa_stream* h, void* stream) {
   // metadata: all -1 (empty slots, no eviction); counters rewritten per append
   cudaError_t e = cudaMemsetAsync(h->meta0, 0xff, h->meta_stride * h->cfg.num_layers, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->store0, 0, 2 * h->store_bytes * h->cfg.num_layers, st);
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(h->split_cnt, 0, static_cast<size_t>(h->cfg.heads) * qpairs_per_frame(h->cfg.P) * 4, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
   for (int l = 0; l < h->cfg.num_layers; ++l) {
     // header counters start at zero (frames, evicted, specials) and -1 (last evicted)
@@ -904,15 +897,18 @@ extern "C" swa_status swa_stream_append_evict_pre_rope3d(swa_stream* h, int glob
 
 namespace {
 
-// split count for the streaming attend: enough CTAs to cover the SMs in few
-// waves while keeping the partial traffic small
+// split count for the streaming attend, in units of one pair's key tile: each
+// wave of CTAs costs its key tiles plus about 8 tiles of start-up and epilogue
+// (measured on B200 at 8 scale + 64 window frames of 1004 tokens: 443, 420 and
+// 460 us for 4, 9 and 16 splits fit 1.45 us per tile and 12.5 us per wave), and
+// every split adds a little to the combine
 int choose_splits(int T, int items_per_split, int max_splits, int sms) {
   int best = 1;
   double best_cost = 1e300;
   for (int k = 1; k <= max_splits && k <= T; ++k) {
     const int64_t ctas = static_cast<int64_t>(items_per_split) * k;
     const int64_t waves = (ctas + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) * cdiv(T, k) + (k > 1 ? 2.0 + 0.25 * k : 0.0);
+    const double cost = static_cast<double>(waves) * (cdiv(T, k) + 8) + (k > 1 ? 0.25 * k : 0.0);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = k;
@@ -974,7 +970,6 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   p.out = out;
   p.part_o = h->part_o;
   p.part_ml = h->part_ml;
-  p.split_cnt = h->split_cnt;
   p.seg_row = seg_row;
   p.seg_len = seg_len;
   p.meta_hdr = hdr;
@@ -991,8 +986,11 @@ swa_status stream_attend_impl(swa_stream* h, int global_idx, const void* q_frame
   p.scale_log2 = scale_log2(c.head_dim);
   cudaError_t e = launch_attn_tc(p, c.head_dim, static_cast<int64_t>(items) * splits, st);
   if (e != cudaSuccess) return SWA_ERR_CUDA;
-  // splits > 1: the last CTA of each work item merges the item's partials
-  return cuda_status(e);
+  if (splits == 1) return SWA_OK;  // every item wrote its rows of out itself
+  // the combine merges the splits, launched behind the attend so that its CTAs are
+  // resident and waiting when the attend's last wave ends
+  const int64_t out_ld = q_ld ? q_ld : static_cast<int64_t>(c.heads) * c.head_dim;
+  return cuda_status(launch_combine(h->part_o, h->part_ml, out, c.P, c.heads, splits, c.head_dim, out_ld, q_h0, st));
 }
 }  // namespace
 

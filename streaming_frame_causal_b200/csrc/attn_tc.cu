@@ -1,7 +1,7 @@
 // attn_tc.cu -- tcgen05 / TMEM / TMA attention kernel for sm_100a (bf16 in,
 // f32 accumulate, bf16 out), used by the frame-causal prefill, the streaming
-// attend (split-KV, merged by the last CTA of each work item) and the
-// token-band GQA prefill.
+// attend (split-KV; combine_kernel, launched behind it, merges the splits) and
+// the token-band GQA prefill.
 //
 // What it computes: O = softmax(Q K^T / sqrt(D)) V over the keys the schedule
 // lists for a 128-row query tile ("Sliding Window Attention Mechanism in
@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // a split stream attend's combine (programmatic launch) may launch now; it waits
+  // for this grid before it reads a partial
+  griddep_launch_dependents();
 
   const Work w = decode_work(p);
   const int T = w.t_end - w.t_begin;
@@ -760,78 +763,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     } else if (T == 0 && w.split >= 0 && (g == 0 || has_b) && r < my_rows) {
-      // empty split: contributes nothing to the merge
+      // empty split: contributes nothing to the combine
       const int row = my_row0 + r;
       const int64_t idx = (static_cast<int64_t>(w.split) * p.Nq + row) * p.Hq + my_h;
       p.part_ml[idx * 2 + 0] = -INFINITY;
       p.part_ml[idx * 2 + 1] = 0.f;
-    }
-    if (w.split >= 0) {
-      // ---- split-KV merge in the item's last CTA: every thread publishes its
-      // partial stores (fence), the 256 softmax threads meet, one of them
-      // counts this CTA in; the CTA that completes the count merges all of the
-      // item's partials, O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c (m
-      // in log2 units), and puts the count back for the next launch
-      volatile int* flag = reinterpret_cast<volatile int*>(gbase + PL::kOffTmem + 8);
-      const int item = static_cast<int>(blockIdx.x % (static_cast<unsigned>(p.Hq) * p.n_pairs));
-      __threadfence();
-      __syncwarp();
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (warp == 4 && lane == 0) *flag = (atomicAdd(p.split_cnt + item, 1) == p.splits - 1) ? 1 : 0;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (*flag) {
-        __threadfence();
-        if ((g == 0 || has_b) && r < my_rows) {
-          const int row = my_row0 + r;
-          const int64_t stride = static_cast<int64_t>(p.Nq) * p.Hq;
-          const int64_t base_idx = static_cast<int64_t>(row) * p.Hq + my_h;
-          float M = -INFINITY;
-#pragma unroll 4
-          for (int c = 0; c < p.splits; ++c) M = fmaxf(M, __ldcg(p.part_ml + (c * stride + base_idx) * 2));
-          float L = 0.f;
-#pragma unroll 4
-          for (int c = 0; c < p.splits; ++c) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (c * stride + base_idx) * 2));
-            L = fmaf((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M), ml.y, L);
-          }
-          const float inv = 1.f / L;
-          const int64_t out_ld = p.out_ld ? p.out_ld : static_cast<int64_t>(p.Hq) * D;
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * out_ld +
-                               static_cast<int64_t>(p.out_h0 + my_h) * D;
-          // 32 output columns at a time, each the weighted sum over the splits
-          // (four splits' loads in flight at once)
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            float o[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0.f;
-#pragma unroll 4
-            for (int c = 0; c < p.splits; ++c) {
-              const float m_c = __ldcg(p.part_ml + (c * stride + base_idx) * 2);
-              const float wc = (m_c == -INFINITY) ? 0.f : exp2f(m_c - M);
-              const float4* src = reinterpret_cast<const float4*>(p.part_o + (c * stride + base_idx) * D + c0);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float4 v = __ldcg(src + e);
-                o[4 * e] = fmaf(wc, v.x, o[4 * e]);
-                o[4 * e + 1] = fmaf(wc, v.y, o[4 * e + 1]);
-                o[4 * e + 2] = fmaf(wc, v.z, o[4 * e + 2]);
-                o[4 * e + 3] = fmaf(wc, v.w, o[4 * e + 3]);
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 v;
-              v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
-              v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
-              v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
-              v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + c0 + e) = v;
-            }
-          }
-        }
-        if (warp == 4 && lane == 0) p.split_cnt[item] = 0;
-      }
     }
   }
 
@@ -845,6 +781,87 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- combine
+// O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c  (m in log2 units), the
+// log-sum-exp merge of split-KV partials.  One warp per (row, head): lane c
+// holds split c's (m, l), the warp reduces M and the weighted sum, then every
+// lane accumulates its slice of O over the splits with independent loads.
+namespace {
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part_o,
+                                                      const float* __restrict__ part_ml,
+                                                      __nv_bfloat16* __restrict__ out, int rows,
+                                                      int H, int splits, int64_t out_ld, int out_h0) {
+  griddep_wait();  // behind the attend (programmatic launch): its partials first
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows * H) return;
+  const int64_t stride = static_cast<int64_t>(rows) * H;
+  float mc = -INFINITY, lc = 0.f;
+  if (lane < splits) {
+    const float2 ml = *reinterpret_cast<const float2*>(part_ml + (lane * stride + gw) * 2);
+    mc = ml.x;
+    lc = ml.y;
+  }
+  float M = mc;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float wc = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+  float L = wc * lc;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  constexpr int E = D / 32;  // elements per lane: 2 (D = 64) or 4 (D = 128)
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int c = 0; c < splits; ++c) {
+    const float w = __shfl_sync(0xffffffffu, wc, c);
+    const float* src = part_o + (c * stride + gw) * D + lane * E;
+    if constexpr (E == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+    } else {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    }
+  }
+  const float inv = 1.f / L;
+  const int row = gw / H, h = gw - row * H;
+  __nv_bfloat16* dst = out + static_cast<int64_t>(row) * out_ld + static_cast<int64_t>(out_h0 + h) * D + lane * E;
+  if constexpr (E == 2) {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  } else {
+    uint2 v;
+    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = v;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H, int splits,
+                           int head_dim, int64_t out_ld, int out_h0, cudaStream_t stream) {
+  if (splits < 1 || splits > 32) return cudaErrorInvalidValue;  // one split per lane
+  const dim3 blocks(static_cast<unsigned>((static_cast<int64_t>(rows) * H + 7) / 8));
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  cudaError_t e;
+  if (head_dim == 64)
+    e = launch_after(combine_kernel<64>, blocks, dim3(256), 0, stream, part_o, part_ml, o, rows, H, splits,
+                     out_ld, out_h0);
+  else if (head_dim == 128)
+    e = launch_after(combine_kernel<128>, blocks, dim3(256), 0, stream, part_o, part_ml, o, rows, H, splits,
+                     out_ld, out_h0);
+  else
+    return cudaErrorInvalidValue;
+  count_launches(1);
+  return e;
+}
 
 int tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? Plan<64>::kSmemBytes : head_dim == 128 ? Plan<128>::kSmemBytes : -1;

@@ -43,14 +43,16 @@ struct TcParams {
   int W, n_qtiles;           // band mode
   int splits, max_segs;      // stream mode
   float scale_log2;          // log2(e) / sqrt(D)
-  int* split_cnt;            // stream mode, splits > 1: per work item (head, query-tile pair),
-                             // CTAs that have written their partials; the last one merges
-                             // them into out and puts the count back to 0
   int64_t out_ld;            // elements between consecutive token rows of out (0: Hq * D)
   int out_h0;                // head of out that query head 0 writes (a head slice of wider rows)
 };
 
 cudaError_t launch_attn_tc(const TcParams& p, int head_dim, int64_t n_items, cudaStream_t stream);
+// merge ``splits`` (<= 32) split-KV partials [splits, rows, H, D] into bf16 out rows
+// out_ld elements apart (heads from out_h0); a programmatic launch that waits for
+// the attend ahead of it on the stream
+cudaError_t launch_combine(const float* part_o, const float* part_ml, void* out, int rows, int H, int splits,
+                           int head_dim, int64_t out_ld, int out_h0, cudaStream_t stream);
 int tc_smem_bytes(int head_dim);
 
 // ---------------------------------------------------------------- SIMT f32 path
