@@ -817,6 +817,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   for (int c = 0; c < splits; ++c) {
     const float w = __shfl_sync(0xffffffffu, wc, c);
+    if (w == 0.f) continue;  // a split without keys: its O was never written
     const float* src = part_o + (c * stride + gw) * D + lane * E;
     if constexpr (E == 2) {
       const float2 v = *reinterpret_cast<const float2*>(src);
