@@ -96,6 +96,15 @@ int64_t swa_sched_prefill(int B, int S, int P, int heads, int sliding_window_siz
  * SWA_ERR_ARG. */
 int swa_sched_decode(int B, int Hkv, int W, long long pos, int sms, int32_t* out);
 
+/* swa_sched_stream: the launch swa_stream_attend makes for ``key_tiles`` 128-token
+ * key tiles (the key runs of the retained frames and specials, each cut into whole
+ * tiles), ``heads`` heads, frames of ``P`` tokens, cfg.max_splits = ``max_splits``
+ * and ``sms`` SMs.  The (query-tile pair, head) items are each cut into ``splits``
+ * contiguous key-tile ranges, one CTA each; a combine kernel merges the splits when
+ * there is more than one.  out[4] = {splits, CTAs, fewest and most key tiles of a
+ * split}.  Returns SWA_OK or SWA_ERR_ARG. */
+int swa_sched_stream(int key_tiles, int heads, int P, int max_splits, int sms, int32_t* out);
+
 /* ---------------------------------------------------------------- prefill
  * Frame-causal sliding-window attention over a whole clip ([AGG], [IO]).
  *   q, k, v, out: [B, S*P, heads, head_dim] contiguous, i.e. the pages'

@@ -67,6 +67,7 @@ _sigs = {
     "swa_sched_frame_intervals": (_i, [_i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i)]),
     "swa_sched_prefill": (_i64, [_i, _i, _i, _i, _i, _i, _i, _vp, _i64]),
     "swa_sched_decode": (_i, [_i, _i, _i, C.c_longlong, _i, _vp]),
+    "swa_sched_stream": (_i, [_i, _i, _i, _i, _i, _vp]),
     "swa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "swa_prefill_heads": (_i, [_vp, _vp, _vp, _vp] + [_i] * 11 + [_vp]),
     "swa_stream_append_evict_heads": (_i, [_vp, _i, _i, _vp, _vp, _i, _i, _vp]),
@@ -177,6 +178,13 @@ def swa_sched_decode(B: int, Hkv: int, W: int, pos: int, sms: int = 148) -> dict
     out = (C.c_int * 5)()
     _check(_lib.swa_sched_decode(B, Hkv, W, pos, sms, out), "swa_sched_decode")
     return {"pieces": out[0], "piece_len": out[1], "grid": out[2], "slots": out[3], "n_valid": out[4]}
+
+
+def swa_sched_stream(key_tiles: int, heads: int, P: int, max_splits: int = 12, sms: int = 148) -> dict:
+    """The streaming attend's launch plan (see include/swa.h)."""
+    out = (C.c_int * 4)()
+    _check(_lib.swa_sched_stream(key_tiles, heads, P, max_splits, sms, out), "swa_sched_stream")
+    return {"splits": out[0], "ctas": out[1], "min_tiles": out[2], "max_tiles": out[3]}
 
 
 # ---------------------------------------------------------------- prefill

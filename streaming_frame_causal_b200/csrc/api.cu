@@ -251,6 +251,29 @@ extern "C" int64_t swa_sched_prefill(int B, int S, int P, int heads, int sliding
   return n;
 }
 
+namespace {
+int choose_splits(int T, int items_per_split, int max_splits, int sms);
+}
+
+extern "C" int swa_sched_stream(int key_tiles, int heads, int P, int max_splits, int sms, int32_t* out) {
+  if (key_tiles < 1 || heads < 1 || P < 1 || max_splits < 1 || max_splits > 32 || sms < 1 || !out)
+    return SWA_ERR_ARG;
+  const int items = heads * qpairs_per_frame(P);
+  const int splits = choose_splits(key_tiles, items, max_splits, sms);
+  int lo = key_tiles, hi = 0;  // fewest and most key tiles of a split
+  for (int s = 0; s < splits; ++s) {
+    int t0, t1;
+    split_range(key_tiles, splits, s, &t0, &t1);
+    lo = imin(lo, t1 - t0);
+    hi = imax(hi, t1 - t0);
+  }
+  out[0] = splits;
+  out[1] = items * splits;
+  out[2] = lo;
+  out[3] = hi;
+  return SWA_OK;
+}
+
 extern "C" int swa_sched_decode(int B, int Hkv, int W, long long pos, int sms, int32_t* out) {
   if (B < 1 || Hkv < 1 || W < 1 || pos < 0 || sms < 1 || !out) return SWA_ERR_ARG;
   const int n_valid = (pos >= W - 1) ? W : static_cast<int>(pos + 1);

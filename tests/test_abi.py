@@ -190,6 +190,30 @@ def test_decode_plan_bench_shape_and_bad_args(swa):
             swa.swa_sched_decode(*bad)
 
 
+@pytest.mark.parametrize("T,H,P,max_splits", [(576, 16, 1004, 12), (601, 16, 1004, 12), (576, 8, 1004, 12),
+                                               (576, 16, 1004, 32), (8, 2, 200, 12), (3, 2, 130, 12),
+                                               (1, 1, 21, 12), (576, 16, 1004, 1)])
+def test_stream_plan_splits_every_item_into_nonempty_ranges(swa, T, H, P, max_splits):
+    """The streaming attend's split count stays within the handle's partial
+    buffers, never exceeds the key tiles (no split is empty, so the combine never
+    reads an unwritten partial), and the ranges differ by at most one tile."""
+    pl = swa.swa_sched_stream(T, H, P, max_splits)
+    n_pairs = -(-(-(-P // 128)) // 2)
+    assert 1 <= pl["splits"] <= min(max_splits, T)
+    assert pl["ctas"] == H * n_pairs * pl["splits"]
+    assert pl["min_tiles"] >= 1 and pl["max_tiles"] - pl["min_tiles"] <= 1
+
+
+def test_stream_plan_bench_shape_and_bad_args(swa):
+    # 8 scale + 64 window frames of 1004 tokens, 16 heads: nine splits of 64 key tiles
+    # (576 CTAs, 3.9 waves on 148 SMs), also with room for 32 (4 and 16 ran slower)
+    assert swa.swa_sched_stream(576, 16, 1004, 12) == {"splits": 9, "ctas": 576, "min_tiles": 64, "max_tiles": 64}
+    assert swa.swa_sched_stream(576, 16, 1004, 32)["splits"] == 9
+    for bad in ((0, 16, 1004, 12), (576, 0, 1004, 12), (576, 16, 0, 12), (576, 16, 1004, 0), (576, 16, 1004, 33)):
+        with pytest.raises(swa.SwaError):
+            swa.swa_sched_stream(*bad)
+
+
 def test_head_slices_and_generated_rope_are_validated(swa):
     lib = swa._lib
     # row stride shorter than head0 + heads: rejected before anything runs
