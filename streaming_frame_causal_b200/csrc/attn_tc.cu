@@ -70,6 +70,7 @@ constexpr int kRegsSoftmax = 216; // warpgroups 1-2 (softmax) after setmaxnreg.i
 static_assert(4 * kRegsCtl + 8 * kRegsSoftmax <= 12 * kRegsLaunch,
               "register split must fit the pool the CTA was launched with");
 constexpr int kRows = kTileRows;       // 128
+constexpr int kMaxSegSmem = 1024;      // key runs whose tile prefix a CTA keeps in shared memory
 constexpr int kSubBytes = 128 * 128;   // one 128-row x 64-column bf16 sub-tile (16 KB)
 
 template <int D>
@@ -109,8 +110,9 @@ struct Plan {
   static constexpr int kOffOnes = kOffV + kStages * kTileBytes;  // the constant block (kSumCol)
   static constexpr int kOffBar = kOffOnes + (kSumCol ? kSubBytes : 0);
   static constexpr int kNumBars = 2 + 4 * kStages + 3 + 2 + 2 + 2 + 2 + 2;
-  static constexpr int kOffTmem = kOffBar + kNumBars * 8;   // TMEM base (4 bytes), then the merge flag
-  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;   // TMEM base (4 bytes)
+  static constexpr int kOffSeg = kOffTmem + 16;              // stream mode: key tiles before each run
+  static constexpr int kSmemBytes = kOffSeg + kMaxSegSmem * 4 + 1024;  // + alignment slack
 };
 
 struct Work {
@@ -124,6 +126,7 @@ struct Work {
   int srow0, slen0, srow1, slen1;  // inline key runs (frame and band modes)
   const int* grow;                 // key runs in device metadata (stream mode)
   const int* glen;
+  const int* tpre;                 // stream mode: key tiles before run s (shared memory), or null
   SWA_DEV int seg_row(int s) const { return grow ? __ldg(grow + s) : (s == 0 ? srow0 : srow1); }
   SWA_DEV int seg_len(int s) const { return glen ? __ldg(glen + s) : (s == 0 ? slen0 : slen1); }
 };
@@ -135,6 +138,20 @@ struct Cursor {
 SWA_DEV bool cursor_seek(const Work& w, int t, Cursor& c) {
   c.s = 0;
   c.off = 0;
+  if (w.tpre) {
+    // run s holds key tiles tpre[s] .. tpre[s+1]-1: binary search, no walk over
+    // the runs in global memory
+    if (t < 0 || t >= w.tpre[w.nseg]) return false;
+    int lo = 0, hi = w.nseg;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (w.tpre[mid] <= t) lo = mid;
+      else hi = mid;
+    }
+    c.s = lo;
+    c.off = (t - w.tpre[lo]) * kRows;
+    return true;
+  }
   while (c.s < w.nseg) {
     const int n = cdiv(w.seg_len(c.s), kRows);
     if (t < n) {
@@ -167,10 +184,11 @@ SWA_DEV int total_tiles(const Work& w) {
   return T;
 }
 
-SWA_DEV Work decode_work(const TcParams& p) {
+SWA_DEV Work decode_work(const TcParams& p, const int* tpre) {
   Work w;
   w.grow = nullptr;
   w.glen = nullptr;
+  w.tpre = nullptr;
   w.split = -1;
   w.nseg = 0;
   w.srow0 = w.slen0 = w.srow1 = w.slen1 = 0;
@@ -227,7 +245,8 @@ SWA_DEV Work decode_work(const TcParams& p) {
     w.glen = p.seg_len;
     const int n = __ldg(p.meta_hdr + 5);
     w.nseg = (n >= 0 && n <= p.max_segs) ? n : 0;
-    const int T = total_tiles(w);
+    if (w.nseg < kMaxSegSmem) w.tpre = tpre;
+    const int T = w.tpre ? w.tpre[w.nseg] : total_tiles(w);
     split_range(T, p.splits, it.split, &w.t_begin, &w.t_end);
     w.split = (p.splits > 1) ? it.split : -1;
   }
@@ -268,10 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // a split stream attend's combine (programmatic launch) may launch now; it waits
   // for this grid before it reads a partial
   griddep_launch_dependents();
-
-  const Work w = decode_work(p);
-  const int T = w.t_end - w.t_begin;
-  const bool has_b = w.rows1 > 0;
 
   // barriers
   const uint32_t bar0 = base + PL::kOffBar;
@@ -336,10 +351,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     fence_proxy_async_smem();
   }
+  int* tpre = reinterpret_cast<int*>(gbase + PL::kOffSeg);
+  if (p.mode == TC_STREAM && warp == 2) {
+    // the tiles of the key runs, summed into a prefix in shared memory by one warp
+    // (128 runs' lengths loaded at a time), so that no thread walks the runs in
+    // global memory to find its split's first tile
+    const int n = __ldg(p.meta_hdr + 5);
+    const int nseg = (n >= 0 && n <= p.max_segs) ? n : 0;
+    if (nseg < kMaxSegSmem) {
+      if (lane == 0) tpre[0] = 0;
+      int carry = 0;
+      for (int c0 = 0; c0 < nseg; c0 += 128) {
+        int v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int sg = c0 + 32 * k + lane;
+          v[k] = sg < nseg ? cdiv(__ldg(p.seg_len + sg), kRows) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v[k], off);
+            if (lane >= off) v[k] += y;
+          }
+          const int sg = c0 + 32 * k + lane;
+          if (sg < nseg) tpre[sg + 1] = carry + v[k];
+          carry += __shfl_sync(0xffffffffu, v[k], 31);
+        }
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + PL::kOffTmem);
+  const Work w = decode_work(p, tpre);
+  const int T = w.t_end - w.t_begin;
+  const bool has_b = w.rows1 > 0;
   if (warp < 4) {
   reg_dealloc<kRegsCtl>();
   if (warp == 0 || warp == 3) {
