@@ -38,24 +38,44 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
   const int64_t special_row0 = static_cast<int64_t>(p.n_slots) * p.ppf * p.page_tokens;
   const bool move_special = (ev >= 0) && p.cross_special;
 
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < 2 * per_tensor;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int tsel = static_cast<int>(idx / per_tensor);
-    const int64_t rem = idx - tsel * per_tensor;
-    const int row = static_cast<int>(rem / chunks);
-    const int ch = static_cast<int>(rem - static_cast<int64_t>(row) * chunks);
-    uint8_t* store = tsel ? p.v_store : p.k_store;
-    const uint8_t* src = tsel ? p.v_src : p.k_src;
-    uint4* dst = reinterpret_cast<uint4*>(store + (slot_row0 + row) * p.row_bytes) + ch;
-    if (move_special && row < p.num_special) {
-      const int64_t sp_row = special_row0 + static_cast<int64_t>(ev - p.S) * p.num_special + row;
-      reinterpret_cast<uint4*>(store + sp_row * p.row_bytes)[ch] = *dst;
+  // 16-byte chunks, four per thread with their loads issued before the stores;
+  // a frame is at most 2^31 chunks, so 32-bit indices
+  const int n = static_cast<int>(2 * per_tensor);
+  const int stride = static_cast<int>(gridDim.x * blockDim.x);
+  for (int base = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); base < n; base += 4 * stride) {
+    uint4 v[4];
+    uint4* dst[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = base + k * stride;
+      dst[k] = nullptr;
+      if (idx >= n) continue;
+      const int tsel = idx >= per_tensor;
+      const int rem = idx - (tsel ? static_cast<int>(per_tensor) : 0);
+      const int row = rem / chunks;
+      const int ch = rem - row * chunks;
+      uint8_t* store = tsel ? p.v_store : p.k_store;
+      dst[k] = reinterpret_cast<uint4*>(store + (slot_row0 + row) * p.row_bytes) + ch;
+      if (move_special && row < p.num_special) {
+        const int64_t sp_row = special_row0 + static_cast<int64_t>(ev - p.S) * p.num_special + row;
+        reinterpret_cast<uint4*>(store + sp_row * p.row_bytes)[ch] = *dst[k];
+      }
+      if (p.copy) {
+        const uint8_t* src = tsel ? p.v_src : p.k_src;
+        v[k] = reinterpret_cast<const uint4*>(src + p.src_off + static_cast<int64_t>(row) * p.src_row_bytes)[ch];
+      }
     }
-    if (p.copy) *dst = reinterpret_cast<const uint4*>(src + p.src_off + static_cast<int64_t>(row) * p.src_row_bytes)[ch];
+    if (p.copy) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (dst[k]) *dst[k] = v[k];
+    }
   }
 
-  if (blockIdx.x != 0) return;
   // ---------------------------------------------------------------- metadata
+  // every thread of the grid takes a share of the page table, the key runs and
+  // the slot map (the table has ~4,500 entries at 72 frames of 63 pages), so no
+  // single block is left with it after the copy
   int* hdr = p.meta;
   int* slot_frame = p.meta + p.off_slot_frame;
   int* pages = p.meta + p.off_page_table;
@@ -70,27 +90,29 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
   const int n_pages = n_ret * p.ppf + sp_pages;
   const int n_segs = n_ret + (n_special > 0 ? 1 : 0);
   if (n_pages > p.max_pages || n_segs > p.max_segs) {
-    if (threadIdx.x == 0) latch_error(p.err, ERR_BAD_META);
+    if (blockIdx.x == 0 && threadIdx.x == 0) latch_error(p.err, ERR_BAD_META);
     return;
   }
+  const int gt = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  const int gn = static_cast<int>(gridDim.x * blockDim.x);
   // retained frame with ordinal o (ascending frame index)
   auto ret_frame = [&](int o) { return o < n_scale ? o : wlo + (o - n_scale); };
-  for (int e = threadIdx.x; e < n_ret * p.ppf; e += blockDim.x) {
+  for (int e = gt; e < n_ret * p.ppf; e += gn) {
     const int o = e / p.ppf;
     const int pg = e - o * p.ppf;
     pages[e] = stream_slot(ret_frame(o), p.S, p.Wc) * p.ppf + pg;
   }
-  for (int e = threadIdx.x; e < sp_pages; e += blockDim.x) pages[n_ret * p.ppf + e] = p.n_slots * p.ppf + e;
-  for (int o = threadIdx.x; o < n_ret; o += blockDim.x) {
+  for (int e = gt; e < sp_pages; e += gn) pages[n_ret * p.ppf + e] = p.n_slots * p.ppf + e;
+  for (int o = gt; o < n_ret; o += gn) {
     seg_row[o] = stream_slot(ret_frame(o), p.S, p.Wc) * p.ppf * p.page_tokens;
     seg_len[o] = p.P;
   }
-  if (threadIdx.x == 0 && n_special > 0) {
+  if (gt == 0 && n_special > 0) {
     seg_row[n_ret] = p.n_slots * p.ppf * p.page_tokens;
     seg_len[n_ret] = n_special;
   }
   // slot map: which frame each slot holds after this append
-  for (int s = threadIdx.x; s < p.n_slots; s += blockDim.x) {
+  for (int s = gt; s < p.n_slots; s += gn) {
     int f = -1;
     if (p.Wc <= 0 || s < p.S) {
       f = (s <= i) ? s : -1;
@@ -103,7 +125,7 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
     }
     slot_frame[s] = f;
   }
-  if (threadIdx.x == 0) {
+  if (gt == 0) {
     hdr[0] = i + 1;
     hdr[1] = n_ev;
     hdr[2] = n_special;
@@ -195,7 +217,8 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t strea
 
 cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
   const int64_t work = 2LL * p.P * (p.row_bytes >> 4);
-  int64_t blocks = (work + 255) / 256;
+  if (work > 0x7fffffffLL) return cudaErrorInvalidValue;  // the kernel indexes chunks in 32 bits
+  int64_t blocks = (work + 1023) / 1024;  // four chunks per thread
   if (blocks < 1) blocks = 1;
   if (blocks > 4096) blocks = 4096;
   append_evict_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
