@@ -7,15 +7,16 @@ input, all inputs resident in HBM:
               frames (schedule + tcgen05 attention)                  1.474 TFLOP
   * stream    8 consecutive frames of a 300-frame-style stream at steady state:
               append + evict on the device, split-KV attend over 8 scale + 64
-              window frames (72 x 1004 keys), merged in-kernel 8 x 0.297 TFLOP
+              window frames (72 x 1004 keys), then the combine   8 x 0.297 TFLOP
   * band      Mistral-style token window: 32768 tokens, GQA 32/8, head_dim 128,
               W = 4096                                               2.062 TFLOP
   * decode    batch 64 at position 200000 against a 4096-slot rolling cache,
               GQA 32/8, head_dim 128 (1 GiB of K/V read)         64 tokens
 Timed apart from the step and reported under ``parts`` as well: the whole
 300-frame stream from an empty cache (fill included, frames/s and per-frame
-latency percentiles), the 1000-frame stream with special-token retention near
-frame 999, the non-keyframe attend, and the attention prologue (with a RoPE
+latency percentiles), the whole 1000-frame stream with special-token retention
+(and its last 8 frames apart), the non-keyframe attend, and the attention
+prologue (with a RoPE
 table and with the 3-D RoPE generated inside it).
 ``value`` is useful attention TFLOP/s over the whole step (visible query-key
 pairs x 4 x head_dim per head; masked and padded work not counted).  Per-stage
