@@ -249,6 +249,18 @@ def test_transient_attend_full_size(swa):
                       at={79, 80}, check_rows=rows, keyframes={79})
 
 
+def test_more_key_runs_than_the_shared_prefix_holds(swa):
+    """No window (every frame retained) over 1030 frames of 16 tokens, 2 x 64:
+    from frame 1023 on the attend sees 1024 or more key runs, more than a CTA
+    keeps the tile prefix of in shared memory, so it walks the runs in the device
+    metadata instead; each pair has a single query tile, and the frame's keys are
+    cut into as many splits as the handle allows.  Bookkeeping bit-exact on every
+    frame; attention against the oracle at frame 0, at frame 1022 (the last whose
+    runs fit the prefix), 1023 and 1029."""
+    _stream(swa, F=1030, P=16, H=2, D=64, S=0, Wc=0, special=False, dtype=torch.bfloat16,
+            frames_to_check={0, 1022, 1023, 1029})
+
+
 def test_camera_only_retention(swa):
     """Evicted frames keep only their camera token (num_special = 1, the reading
     taken for kv_cache_camera_only): bookkeeping bit-exact, attention matches."""
