@@ -144,18 +144,29 @@ __global__ void __launch_bounds__(256) append_evict_kernel(const AppendParams p)
 // the scratch run.  Nothing persistent is written, so the roll-back is free.
 __global__ void __launch_bounds__(256) transient_prepare_kernel(const TransientParams p) {
   const int chunks = p.row_bytes >> 4;
-  const int64_t per_tensor = static_cast<int64_t>(p.P) * chunks;
+  const int per_tensor = p.P * chunks;  // the host keeps 2 * per_tensor below 2^31
   const int64_t row0 = static_cast<int64_t>(p.scratch_page) * p.page_tokens;
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < 2 * per_tensor;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int tsel = static_cast<int>(idx / per_tensor);
-    const int64_t rem = idx - tsel * per_tensor;
-    const int row = static_cast<int>(rem / chunks);
-    const int ch = static_cast<int>(rem - static_cast<int64_t>(row) * chunks);
-    uint8_t* store = tsel ? p.v_store : p.k_store;
-    const uint8_t* src = tsel ? p.v_src : p.k_src;
-    reinterpret_cast<uint4*>(store + (row0 + row) * p.row_bytes)[ch] =
-        reinterpret_cast<const uint4*>(src + static_cast<int64_t>(row) * p.row_bytes)[ch];
+  // 16-byte chunks, four per thread with their loads issued before the stores
+  const int n_chunks = 2 * per_tensor;
+  const int stride = static_cast<int>(gridDim.x * blockDim.x);
+  for (int base = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); base < n_chunks; base += 4 * stride) {
+    uint4 v[4];
+    uint4* dst[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = base + k * stride;
+      dst[k] = nullptr;
+      if (idx >= n_chunks) continue;
+      const int tsel = idx >= per_tensor;
+      const int rem = idx - (tsel ? per_tensor : 0);
+      const int row = rem / chunks;
+      const int ch = rem - row * chunks;
+      dst[k] = reinterpret_cast<uint4*>((tsel ? p.v_store : p.k_store) + (row0 + row) * p.row_bytes) + ch;
+      v[k] = reinterpret_cast<const uint4*>((tsel ? p.v_src : p.k_src) + static_cast<int64_t>(row) * p.row_bytes)[ch];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (dst[k]) *dst[k] = v[k];
   }
   if (blockIdx.x != 0) return;
   const int* hdr = p.meta;
@@ -228,7 +239,8 @@ cudaError_t launch_append_evict(const AppendParams& p, cudaStream_t stream) {
 
 cudaError_t launch_transient_prepare(const TransientParams& p, cudaStream_t stream) {
   const int64_t work = 2LL * p.P * (p.row_bytes >> 4);
-  int64_t blocks = (work + 255) / 256;
+  if (work > 0x7fffffffLL) return cudaErrorInvalidValue;  // the kernel indexes chunks in 32 bits
+  int64_t blocks = (work + 1023) / 1024;  // four chunks per thread
   if (blocks < 1) blocks = 1;
   if (blocks > 4096) blocks = 4096;
   transient_prepare_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
